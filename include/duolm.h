@@ -1,0 +1,228 @@
+/*
+ * duolm.h -- C ABI of the DuoLM multi-item-scoring (MIS) ranker on B200.
+ *
+ * The library scores the K candidates of each request with a Qwen3-style
+ * ranker: request tokens are embedded through a virtual-id lookup, the shared
+ * prefix of each request is computed once, every candidate branch attends to
+ * that prefix and to itself only (tree mask, unified logical position), and a
+ * shared linear head reads one score per candidate.  Sources:
+ *   DuoLM summary page (paper.rainbus.top, "DuoLM:基于语言模型的快速高效个性化推荐框架"),
+ *   sections 核心方法 (ranker and score head s = w^T h), 方法步骤详情 steps 3-5
+ *   (FP16 item table addressed by virtual id V + i; shared prefix prefilled
+ *   once; candidate j sees only the prefix and itself at logical position L_q;
+ *   scores in input order; CUDA Graph replay), 研究动机 (s^MIS = s).
+ *
+ * Conventions for every call:
+ *   - Return 0 on success, a negative DUOLM_E_* code on failure; the text of
+ *     the last failure is in duolm_last_error(ctx).
+ *   - Pointers documented as "host" are read (or written) only during the
+ *     call and stay owned by the caller.  The library owns all device memory
+ *     it allocates and frees it in duolm_destroy.
+ *   - A context is bound to one device and one CUDA stream and is not
+ *     thread-safe: use one context per stream.
+ *   - Calls that return results to host memory synchronise the context's
+ *     stream before returning.
+ */
+#ifndef DUOLM_H
+#define DUOLM_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DUOLM_OK 0
+#define DUOLM_E_ARG (-1)       /* null pointer, bad size, bad mode or descriptor */
+#define DUOLM_E_ID (-2)        /* a token id is negative or >= vocab + table rows */
+#define DUOLM_E_OFFSETS (-3)   /* offsets do not start at 0 or are not non-decreasing */
+#define DUOLM_E_EMPTY (-4)     /* a request with L = 0 or K = 0, or branch_len < 1 */
+#define DUOLM_E_CAPACITY (-5)  /* batch larger than the reserved capacity */
+#define DUOLM_E_CUDA (-6)      /* a CUDA runtime call failed (text in last_error) */
+#define DUOLM_E_DEVICE (-7)    /* a kernel raised the device error flag */
+#define DUOLM_E_STATE (-8)     /* call out of order (no table loaded, nothing prepared) */
+
+#define DUOLM_DTYPE_FP32 0     /* fp32 weights, fp32 arithmetic everywhere */
+#define DUOLM_DTYPE_BF16 1     /* bf16 weights; fp16 tensor-core operands, fp32 accumulate */
+
+#define DUOLM_MODE_MIS 0          /* shared prefix + tree-masked branches */
+#define DUOLM_MODE_INDEPENDENT 1  /* every candidate as its own full sequence */
+
+typedef struct duolm_ctx duolm_ctx;
+
+/* Ranker shape.  Requirements: d % 8 == 0 and d <= 2048; n_q_heads % n_kv_heads
+ * == 0; head_dim even.  FP32 models: head_dim % 32 == 0 and head_dim <= 256.
+ * BF16 models: head_dim == 128, d % 256 == 0, ffn % 128 == 0,
+ * n_q_heads / n_kv_heads in {1, 2, 4}, n_q_heads + 2 * n_kv_heads even.
+ * Violations fail with DUOLM_E_ARG. */
+typedef struct {
+    int n_layers, d, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
+    float rope_theta, rms_eps;
+    int dtype; /* DUOLM_DTYPE_* */
+} duolm_model_desc;
+
+/* Number of weight tensors duolm_model_load expects: 1 + 11 * n_layers + 2. */
+int duolm_weight_count(const duolm_model_desc *desc);
+
+/*
+ * Create a context on `device` and copy the ranker weights to it.
+ * host_weights: duolm_weight_count(desc) host pointers, each to a row-major
+ *   tensor of the descriptor's dtype (uint16 bfloat16 bit patterns for BF16,
+ *   float for FP32), in this order:
+ *     embed [vocab][d];
+ *     per layer: attn_norm [d], wq [n_q_heads*head_dim][d],
+ *       wk [n_kv_heads*head_dim][d], wv [n_kv_heads*head_dim][d],
+ *       q_norm [head_dim], k_norm [head_dim], wo [d][n_q_heads*head_dim],
+ *       mlp_norm [d], w_gate [ffn][d], w_up [ffn][d], w_down [d][ffn];
+ *     final_norm [d], head [d].
+ *   Matrices are [out_features][in_features].
+ * cuda_stream: a cudaStream_t to run on, or NULL for a stream owned by the
+ *   context.
+ * For BF16 weights each matrix is stored on the device as FP16 times a
+ * power-of-two scale chosen per matrix so that every bfloat16 value converts
+ * exactly; a matrix that cannot be converted exactly fails with DUOLM_E_ARG.
+ * On success *out holds the context; on failure *out is NULL.
+ */
+int duolm_model_load(const duolm_model_desc *desc, const void *const *host_weights, int device,
+                     void *cuda_stream, duolm_ctx **out);
+
+/*
+ * Replace the virtual-id item table D with host FP16 rows (uint16 IEEE
+ * binary16 bit patterns), row-major [n_items][d].  Ranker id vocab + i then
+ * reads row i (DuoLM summary page, 方法步骤详情 step 3).  Synchronous.
+ */
+int duolm_vid_table_load(duolm_ctx *ctx, const uint16_t *fp16_rows, int64_t n_items);
+
+/*
+ * Build the item table on the device from raw encoder outputs through the
+ * continuous interface z_i = e^gamma * rho * a_i / RMS(a_i), RMS without
+ * epsilon, computed in fp64 and rounded to FP16 to nearest even (DuoLM
+ * summary page, 前置知识 "连续输入接口" and 核心方法).
+ * a_rows: host float [n_items][d].  Synchronous.
+ */
+int duolm_vid_table_build(duolm_ctx *ctx, const float *a_rows, int64_t n_items, double gamma,
+                          double rho);
+
+/* Reference scale rho of the interface estimated from the loaded embedding:
+ * the mean over vocabulary rows of each row's RMS, in fp64.  Synchronous. */
+int duolm_embedding_rho(duolm_ctx *ctx, double *rho_out);
+
+/*
+ * Reserve device workspace for batches of up to max_tokens packed tokens,
+ * max_requests requests and max_candidates candidates (after expansion:
+ * independent mode turns each candidate into a request of one candidate).
+ * Optional: duolm_prepare grows the workspace on demand, which frees and
+ * reallocates device memory and re-captures the CUDA graph.
+ */
+int duolm_reserve(duolm_ctx *ctx, int64_t max_tokens, int64_t max_requests, int64_t max_candidates);
+
+/*
+ * Validate and stage one batch.  Request q has prefix
+ * prefix_ids[prefix_offsets[q] .. prefix_offsets[q+1]) (L_q >= 1 tokens) and
+ * candidates cand_offsets[q] .. cand_offsets[q+1]) (K_q >= 1); candidate c
+ * has branch tokens branch_ids[c*branch_len .. (c+1)*branch_len), the last of
+ * which is scored.  All pointers are host; offsets have n_requests + 1
+ * entries and start at 0.  mode is DUOLM_MODE_*.
+ * The packed layout, position ids and attention work list are built on the
+ * host and copied to the device on the context stream (asynchronously: the
+ * host buffers may be reused as soon as the call returns).
+ * In independent mode the batch must fit the reserved capacity after
+ * expansion (K_q * (L_q + b) tokens per request); otherwise DUOLM_E_CAPACITY.
+ */
+int duolm_prepare(duolm_ctx *ctx, int n_requests, const int32_t *prefix_ids,
+                  const int64_t *prefix_offsets, const int32_t *branch_ids,
+                  const int64_t *cand_offsets, int branch_len, int mode);
+
+/*
+ * Run the ranker on the prepared batch, asynchronously on the context
+ * stream.  Scores (fp32, one per candidate, input order) land in the device
+ * buffer returned by duolm_scores_device.  Uses the CUDA graph unless
+ * disabled with duolm_set_graph(ctx, 0).
+ */
+int duolm_execute(duolm_ctx *ctx);
+
+/* Device pointer to the scores of the last duolm_execute ([n_candidates] fp32). */
+const float *duolm_scores_device(const duolm_ctx *ctx);
+
+/* Synchronise the context stream and check the device error flag. */
+int duolm_sync(duolm_ctx *ctx);
+
+/*
+ * One whole call: prepare + execute + copy the scores to host memory
+ * (scores_out: host float [cand_offsets[n_requests]]) + synchronise.
+ */
+int duolm_score(duolm_ctx *ctx, int n_requests, const int32_t *prefix_ids,
+                const int64_t *prefix_offsets, const int32_t *branch_ids,
+                const int64_t *cand_offsets, int branch_len, int mode, float *scores_out);
+
+/* Launch through a captured CUDA graph (1, default) or kernel by kernel (0). */
+int duolm_set_graph(duolm_ctx *ctx, int enabled);
+
+/* Number of kernel launches one duolm_execute issues for the prepared batch
+ * (graph nodes when the graph is used). */
+int64_t duolm_launches_per_execute(const duolm_ctx *ctx);
+
+/* Text of the last failure on this context ("" if none).  Valid until the
+ * next call on the context.  With ctx == NULL: the reason the calling
+ * thread's last duolm_model_load failed. */
+const char *duolm_last_error(const duolm_ctx *ctx);
+
+/* Free every device resource of the context (NULL is ignored). */
+void duolm_destroy(duolm_ctx *ctx);
+
+/* ---- introspection (tests) --------------------------------------------- */
+
+/* Packed layout of the prepared batch as the device holds it: n_tokens,
+ * and per token its ranker id and position id (host int32 [n_tokens] each;
+ * either may be NULL).  Synchronous. */
+int duolm_debug_layout(duolm_ctx *ctx, int64_t *n_tokens, int32_t *ids_out, int32_t *pos_out);
+
+/* Evaluate, on the device, the attention kernels' visibility predicate for
+ * every (query token, key token) pair of request q of the prepared batch:
+ * out is host uint8 [T_q][T_q], T_q = L_q + K_q * b.  Synchronous. */
+int duolm_debug_mask(duolm_ctx *ctx, int request, uint8_t *out);
+
+/* Run the embedding and the first n_layers layers of the prepared batch and
+ * copy the fp32 residual stream out (host float [n_tokens][d]).  n_layers = 0
+ * gives the looked-up rows.  Synchronous. */
+int duolm_debug_residual(duolm_ctx *ctx, int n_layers, float *x_out);
+
+/* Copy the device item table out (host uint16 [n_items][d]).  Synchronous. */
+int duolm_debug_table(duolm_ctx *ctx, uint16_t *out, int64_t n_items);
+
+/* Bytes the last duolm_prepare copied host -> device (the packed plan). */
+int64_t duolm_plan_bytes(const duolm_ctx *ctx);
+
+/*
+ * One projection of layer `layer` through the tensor-core GEMM alone
+ * (BF16 models only): out = a * W^T with W = wqkv (which 0, [qd+2kd][d]),
+ * wo (1, [d][qd]), gate/up (2, [2*ffn][d], rows in 128-row blocks alternating
+ * gate and up) or w_down (3, [d][ffn]).  a: host uint16 fp16 bit patterns
+ * [n_tokens][K] where n_tokens is the prepared batch's token count; out: host
+ * float [n_tokens][N].  Overwrites the batch's activations.  Synchronous.
+ */
+int duolm_debug_gemm(duolm_ctx *ctx, int layer, int which, const uint16_t *a, float *out);
+
+/* Kernel classes of duolm_profile. */
+#define DUOLM_PROF_EMBED 0
+#define DUOLM_PROF_GEMM_QKV 1
+#define DUOLM_PROF_ATTENTION 2
+#define DUOLM_PROF_GEMM_O 3
+#define DUOLM_PROF_RMSNORM 4
+#define DUOLM_PROF_GEMM_GATE_UP 5
+#define DUOLM_PROF_GEMM_DOWN 6
+#define DUOLM_PROF_HEAD 7
+#define DUOLM_PROF_N 8
+
+/*
+ * Run the prepared batch n_steps times kernel by kernel with a CUDA event
+ * after every launch, and return per kernel class the summed device time in
+ * ms (ms_out[DUOLM_PROF_N]) and the number of launches (count_out).
+ * Synchronous; the scores of the last step are left as by duolm_execute.
+ */
+int duolm_profile(duolm_ctx *ctx, int n_steps, double *ms_out, int64_t *count_out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DUOLM_H */

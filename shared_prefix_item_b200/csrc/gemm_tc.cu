@@ -1,0 +1,388 @@
+// Projection GEMMs of the ranker on 5th-generation tensor cores (sm_100a).
+//
+// C[M, N] = A[M, K] * B[N, K]^T with fp16 operands and fp32 accumulation in
+// tensor memory.  One persistent CTA per SM, 192 threads, warp-specialised:
+//   warp 0      TMA producer: streams 128x64 A and BNx64 B tiles (128-byte
+//               swizzle, no multicast) into a STAGES-deep shared-memory ring;
+//   warp 1      allocates 2*BN TMEM columns; lane 0 issues tcgen05.mma
+//               (128 x BN x 16 per instruction) and commits to mbarriers;
+//   warps 2-5   epilogue: each thread owns one accumulator row (TMEM lane),
+//               reads it with tcgen05.ld and applies a fused epilogue.
+// Two accumulator buffers let the epilogue of tile i overlap the mainloop of
+// tile i+1.  Every mbarrier wait is bounded (see common.cuh).
+#include <cstdio>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace duolm {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;  // one 128-byte swizzle row of fp16
+constexpr int kThreads = 192;
+
+template <int BN>
+struct TcCfg {
+  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int A_BYTES = kBM * kBK * 2;
+  static constexpr int B_BYTES = BN * kBK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  static constexpr int SMEM = BAR_OFF + 256 + 1024;  // barriers + alignment slack
+  static constexpr uint32_t TMEM_COLS = 2 * BN;
+  static constexpr uint32_t IDESC = idesc_f16_f32(kBM, BN);
+};
+
+// ---------------------------------------------------------------------------
+// fused epilogues.  `taddr` addresses this thread's row, column 0 of the tile's
+// accumulator; all lanes of the warp must execute the TMEM loads.
+// ---------------------------------------------------------------------------
+struct EpiResid {
+  EpiResidArgs a;
+  template <int BN>
+  __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, bool row_ok, const PlanHdr*, DevStatus*) const {
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      float v[32];
+      tmem_ld32(taddr + c, v);
+      if (row_ok) {
+        float4* p = reinterpret_cast<float4*>(a.x + (int64_t)row * a.ldx + n0 + c);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float4 t = p[j];
+          t.x += v[4 * j + 0] * a.scale;
+          t.y += v[4 * j + 1] * a.scale;
+          t.z += v[4 * j + 2] * a.scale;
+          t.w += v[4 * j + 3] * a.scale;
+          p[j] = t;
+        }
+      }
+    }
+  }
+};
+
+struct EpiSwiglu {
+  EpiSwigluArgs a;
+  template <int BN>
+  __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, bool row_ok, const PlanHdr*,
+                                      DevStatus* st) const {
+    constexpr int H = BN / 2;
+    const int out0 = n0 / 2;
+#pragma unroll 1
+    for (int c = 0; c < H; c += 32) {
+      float g[32], u[32];
+      tmem_ld32(taddr + c, g);
+      tmem_ld32(taddr + H + c, u);
+      if (row_ok) {
+        uint32_t packed[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          float h0 = silu(g[2 * j] * a.scale) * (u[2 * j] * a.scale);
+          float h1 = silu(g[2 * j + 1] * a.scale) * (u[2 * j + 1] * a.scale);
+          __half2 hh = __halves2half2(to_half_checked(h0, st, 20), to_half_checked(h1, st, 20));
+          packed[j] = *reinterpret_cast<uint32_t*>(&hh);
+        }
+        uint4* p = reinterpret_cast<uint4*>(a.h + (int64_t)row * a.ldh + out0 + c);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) p[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+      }
+    }
+  }
+};
+
+// Per 128-column head of the fused Q|K|V output: q and k get RMSNorm over the
+// head (QK-norm) and rotate-half RoPE at the token's logical position; v is
+// copied.  q goes to [T][Hq][128], k and v to the per-head KV buffers.
+struct EpiQkv {
+  EpiQkvArgs a;
+  template <int BN>
+  __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, bool row_ok, const PlanHdr* plan,
+                                      DevStatus* st) const {
+    const int* pos_arr = plan_array<int32_t>(plan, plan->off_pos);
+#pragma unroll 1
+    for (int hl = 0; hl < BN / 128; ++hl) {
+      const int gc = n0 + 128 * hl;
+      const uint32_t base = taddr + 128 * hl;
+      if (gc >= a.qd + a.kd) {  // value head
+        const int head = (gc - a.qd - a.kd) >> 7;
+        __half* dst = a.vc + ((int64_t)head * a.kv_rows + row) * 128;
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 32) {
+          float v[32];
+          tmem_ld32(base + c, v);
+          if (row_ok) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              __half2 hh = __halves2half2(to_half_checked(v[2 * j] * a.scale, st, 21),
+                                          to_half_checked(v[2 * j + 1] * a.scale, st, 21));
+              pk[j] = *reinterpret_cast<uint32_t*>(&hh);
+            }
+            uint4* p = reinterpret_cast<uint4*>(dst + c);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) p[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          }
+        }
+        continue;
+      }
+      const bool is_q = gc < a.qd;
+      const int head = is_q ? (gc >> 7) : ((gc - a.qd) >> 7);
+      const float* gain = is_q ? a.gq : a.gk;
+      __half* dst = is_q ? a.q + ((int64_t)row * a.n_q_heads + head) * 128
+                         : a.kc + ((int64_t)head * a.kv_rows + row) * 128;
+      float ss = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < 128; c += 32) {
+        float v[32];
+        tmem_ld32(base + c, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          float t = v[j] * a.scale;
+          ss += t * t;
+        }
+      }
+      const float r = rsqrtf(ss * (1.0f / 128.0f) + a.eps);
+      int p = row_ok ? pos_arr[row] : 0;
+      if (p < 0 || p >= a.max_pos) {
+        if (row_ok) raise_error(st, ERR_BAD_INDEX, 22);
+        p = 0;
+      }
+      const float2* cs = a.rope + (int64_t)p * 64;
+#pragma unroll 1
+      for (int c = 0; c < 64; c += 32) {
+        float x1[32], x2[32];
+        tmem_ld32(base + c, x1);
+        tmem_ld32(base + 64 + c, x2);
+        if (row_ok) {
+          uint32_t o1[16], o2[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            float r1[2], r2[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int i = c + j + e;
+              const float a1 = (x1[j + e] * a.scale * r) * gain[i];
+              const float a2 = (x2[j + e] * a.scale * r) * gain[64 + i];
+              const float2 t = cs[i];
+              r1[e] = a1 * t.x - a2 * t.y;
+              r2[e] = a2 * t.x + a1 * t.y;
+            }
+            __half2 h1 = __floats2half2_rn(r1[0], r1[1]);
+            __half2 h2 = __floats2half2_rn(r2[0], r2[1]);
+            o1[j / 2] = *reinterpret_cast<uint32_t*>(&h1);
+            o2[j / 2] = *reinterpret_cast<uint32_t*>(&h2);
+          }
+          uint4* p1 = reinterpret_cast<uint4*>(dst + c);
+          uint4* p2 = reinterpret_cast<uint4*>(dst + 64 + c);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            p1[j] = make_uint4(o1[4 * j], o1[4 * j + 1], o1[4 * j + 2], o1[4 * j + 3]);
+            p2[j] = make_uint4(o2[4 * j], o2[4 * j + 1], o2[4 * j + 2], o2[4 * j + 3]);
+          }
+        }
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// the kernel
+// ---------------------------------------------------------------------------
+template <int BN, class Epi>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int Kdim,
+                   int N, const PlanHdr* __restrict__ plan, const Epi epi, DevStatus* st) {
+  using C = TcCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = smem_u32(bars + C::STAGES);
+  const uint32_t tfull0 = smem_u32(bars + 2 * C::STAGES);
+  const uint32_t tempty0 = smem_u32(bars + 2 * C::STAGES + 2);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 4);
+
+  // a bounded wait already gave up in an earlier launch: do nothing
+  if (*reinterpret_cast<volatile const uint32_t*>(&st->flags) & ERR_WAIT_TIMEOUT) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int M = plan->n_tokens;
+  const int m_tiles = (M + kBM - 1) / kBM;
+  const int n_tiles = N / BN;
+  const int num_tiles = m_tiles * n_tiles;
+  const int kblocks = Kdim / kBK;
+
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull0 + 8 * a, 1);
+      mbar_init(tempty0 + 8 * a, 128);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int m_blk = tile % m_tiles, n_blk = tile / m_tiles;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, st, 1)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sb = sa + C::A_BYTES;
+          mbar_arrive_expect_tx(full0 + 8 * stage, C::STAGE_BYTES);
+          tma_load_2d(&tmA, sa, full0 + 8 * stage, kb * kBK, m_blk * kBM);
+          tma_load_2d(&tmB, sb, full0 + 8 * stage, kb * kBK, n_blk * BN);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t use = (uint32_t)(local >> 1);
+        if (!mbar_wait(tempty0 + 8 * acc, (use & 1u) ^ 1u, st, 2)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase, st, 3)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            tc_mma_f16(d_tmem, smem_desc_sw128(sa + 32 * k), smem_desc_sw128(sb + 32 * k), C::IDESC,
+                       (kb | k) != 0 ? 1u : 0u);
+          }
+          tc_commit(empty0 + 8 * stage);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) tc_commit(tfull0 + 8 * acc);
+      }
+    }
+  } else {
+    const int q4 = warp & 3;  // TMEM lane quadrant this warp may access
+    int local = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+      const int acc = local & 1;
+      const uint32_t use = (uint32_t)(local >> 1);
+      if (!mbar_wait(tfull0 + 8 * acc, use & 1u, st, 4)) break;
+      tc_fence_after();
+      const int m_blk = tile % m_tiles, n_blk = tile / m_tiles;
+      const int row = m_blk * kBM + q4 * 32 + lane;
+      const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q4 * 32) << 16);
+      epi.template run<BN>(taddr, row, n_blk * BN, row < M, plan, st);
+      tc_fence_before();
+      mbar_arrive(tempty0 + 8 * acc);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static PFN_encodeTiled get_encode() {
+  static PFN_encodeTiled fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_encodeTiled>(p);
+  }
+  return fn;
+}
+
+bool make_tmap_f16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                      uint32_t box_outer, char* err, size_t errlen) {
+  PFN_encodeTiled enc = get_encode();
+  if (!enc) {
+    snprintf(err, errlen, "cuTensorMapEncodeTiled unavailable");
+    return false;
+  }
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(err, errlen, "cuTensorMapEncodeTiled failed (%d): inner %llu outer %llu box %u x %u", (int)r,
+             (unsigned long long)inner, (unsigned long long)outer, box_inner, box_outer);
+    return false;
+  }
+  return true;
+}
+
+int gemm_tc_smem_bytes(int bn) { return bn == 256 ? TcCfg<256>::SMEM : TcCfg<128>::SMEM; }
+
+cudaError_t gemm_tc_setup() {
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(gemm_tc_kernel<256, EpiResid>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                TcCfg<256>::SMEM)) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(gemm_tc_kernel<256, EpiSwiglu>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                TcCfg<256>::SMEM)) != cudaSuccess)
+    return e;
+  return cudaFuncSetAttribute(gemm_tc_kernel<256, EpiQkv>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              TcCfg<256>::SMEM);
+}
+
+cudaError_t gemm_tc_resid(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
+                          EpiResidArgs e, DevStatus* st, int grid, cudaStream_t s) {
+  gemm_tc_kernel<256, EpiResid><<<grid, kThreads, TcCfg<256>::SMEM, s>>>(a, b, K, N, plan, EpiResid{e}, st);
+  return cudaGetLastError();
+}
+cudaError_t gemm_tc_swiglu(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
+                           EpiSwigluArgs e, DevStatus* st, int grid, cudaStream_t s) {
+  gemm_tc_kernel<256, EpiSwiglu><<<grid, kThreads, TcCfg<256>::SMEM, s>>>(a, b, K, N, plan, EpiSwiglu{e}, st);
+  return cudaGetLastError();
+}
+cudaError_t gemm_tc_qkv(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
+                        EpiQkvArgs e, DevStatus* st, int grid, cudaStream_t s) {
+  gemm_tc_kernel<256, EpiQkv><<<grid, kThreads, TcCfg<256>::SMEM, s>>>(a, b, K, N, plan, EpiQkv{e}, st);
+  return cudaGetLastError();
+}
+
+}  // namespace duolm

@@ -1,0 +1,79 @@
+// Launch interfaces of the ranker's kernels (host side).
+#pragma once
+
+#include "common.cuh"
+
+namespace duolm {
+
+// ---- tcgen05 GEMM:  C[M, N] = A[M, K] * B[N, K]^T, fp16 operands, fp32 accumulate.
+// M is the batch's token count, read on the device from the plan.
+
+struct EpiResidArgs {   // x[row][col] += scale * acc  (fp32 residual stream)
+  float* x;
+  int ldx;
+  float scale;
+};
+struct EpiSwigluArgs {  // tile columns [0, BN/2) gate, [BN/2, BN) up -> h = silu(g) * u, fp16
+  __half* h;
+  int ldh;
+  float scale;
+};
+struct EpiQkvArgs {     // per 128-wide head: q/k RMSNorm + RoPE, v copy; fp16 out
+  __half* q;            // [T][n_q_heads][128]
+  __half* kc;           // [n_kv_heads][kv_rows][128]
+  __half* vc;           // [n_kv_heads][kv_rows][128]
+  const float2* rope;   // [max_pos][64] (cos, sin)
+  int64_t kv_rows;
+  int max_pos;
+  const float* gq;      // q_norm gains [128]
+  const float* gk;      // k_norm gains [128]
+  float scale;
+  float eps;
+  int qd, kd, n_q_heads;
+};
+
+bool make_tmap_f16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                      uint32_t box_outer, char* err, size_t errlen);
+int gemm_tc_smem_bytes(int bn);
+cudaError_t gemm_tc_setup();
+cudaError_t gemm_tc_resid(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
+                          EpiResidArgs e, DevStatus* st, int grid, cudaStream_t s);
+cudaError_t gemm_tc_swiglu(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
+                           EpiSwigluArgs e, DevStatus* st, int grid, cudaStream_t s);
+cudaError_t gemm_tc_qkv(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
+                        EpiQkvArgs e, DevStatus* st, int grid, cudaStream_t s);
+
+// ---- fp32 SIMT GEMM (the fp32 path): C = A * B^T, store or residual add.
+cudaError_t gemm_simt(const float* A, const float* B, float* C, int K, int N, int ldc, bool accumulate,
+                      const PlanHdr* plan, int max_rows, cudaStream_t s);
+
+// ---- elementwise and small kernels
+template <typename OutT>
+cudaError_t embed_norm(const PlanHdr* plan, const void* embed, bool embed_bf16, const __half* table,
+                       int64_t n_table, int vocab, int d, const float* gain, float eps, float* x, OutT* xn,
+                       DevStatus* st, int max_rows, cudaStream_t s);
+template <typename OutT>
+cudaError_t rmsnorm_rows(const PlanHdr* plan, const float* x, int d, const float* gain, float eps, OutT* xn,
+                         DevStatus* st, int max_rows, cudaStream_t s);
+cudaError_t score_head(const PlanHdr* plan, const float* x, int d, const float* gain, const float* w, float eps,
+                       float* scores, int max_cand, cudaStream_t s);
+cudaError_t qkv_post_f32(const PlanHdr* plan, const float* qkv, int n_q_heads, int n_kv_heads, int hd,
+                         const float* gq, const float* gk, float eps, const float2* rope, int max_pos, float* q,
+                         float* kc, float* vc, int64_t kv_rows, DevStatus* st, int max_rows, cudaStream_t s);
+cudaError_t swiglu_f32(const PlanHdr* plan, const float* gu, int F, float* h, int max_rows, cudaStream_t s);
+cudaError_t table_build(const float* a, int64_t n, int d, double scale_num, __half* out, cudaStream_t s);
+cudaError_t embed_rho(const void* embed, bool embed_bf16, int64_t vocab, int d, double* row_rms, double* out,
+                      cudaStream_t s);
+cudaError_t debug_mask(const PlanHdr* plan, int request, uint8_t* out, int64_t tq, cudaStream_t s);
+
+// ---- attention
+cudaError_t attention_f16(const PlanHdr* plan, const __half* q, const __half* kc, const __half* vc,
+                          int64_t kv_rows, int n_q_heads, int n_kv_heads, float scale, __half* o, DevStatus* st,
+                          int grid, cudaStream_t s);
+cudaError_t attention_f32(const PlanHdr* plan, const float* q, const float* kc, const float* vc, int64_t kv_rows,
+                          int n_q_heads, int n_kv_heads, int hd, float scale, float* o, int max_rows,
+                          cudaStream_t s);
+int attention_rows_per_item(int group);
+cudaError_t attention_setup();
+
+}  // namespace duolm
