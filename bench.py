@@ -1,0 +1,410 @@
+"""Throughput of the DuoLM multi-item-scoring ranker: candidate scores/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config c64|c1|stress|catalog-c64|catalog-c8|catalog-c1]
+                    [--mode mis|independent] [--no-graph] [--skip-cpu] [--profile-steps N]
+
+One step is one pass of the whole hot path (virtual-id gather, 28 decoder
+layers with shared-prefix tree-masked attention, score head) over one batch
+of synthetic requests.  Default workload: 64 ragged requests of the
+Qwen3-0.6B-shaped ranker with K = 100 candidates each (the configuration the
+pages' headline throughput is quoted on).  Under torchrun every rank scores
+its own batch of the same recipe (requests are independent: weak scaling,
+no data-path collective); the time is the max over ranks.
+
+Prints one JSON line (rank 0).  `value` times device-resident batches
+(duolm_execute replays of the prepared batch); `e2e` times duolm_score from
+host buffers (validation, packing, host->device copy, pass, scores back).
+`--impl reference` times the oracle (plain fp64 CPU code) on the host cores
+instead, one request of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from synth import workloads as W  # noqa: E402
+
+METRIC = "candidate scores/sec on 1 B200 (Qwen3-0.6B shape, K=100) + % of roofline"
+UNIT = "candidate scores/s"
+H100_C64 = 26404.0  # pages' figure: MIS + CUDA Graph, C=64, 100 candidates, 1x H100 (context)
+
+
+def workload(name: str, shard: int) -> W.Workload:
+    if name == "c64":
+        return W.c64(shard=shard)
+    if name == "c1":
+        return W.c1(shard=shard)
+    if name == "stress":
+        return W.stress(shard=shard)
+    if name.startswith("catalog-c"):
+        return W.catalog(int(name[len("catalog-c"):]), shard=shard)
+    raise SystemExit(f"unknown config {name}")
+
+
+def describe(wl: W.Workload, mode: str, graph: bool, n: int) -> dict:
+    Ls = [r.L for r in wl.requests]
+    return {
+        "workload": f"{wl.name}: {len(wl.requests)} requests x K={wl.requests[0].K} candidates, "
+                    f"b={wl.branch_len}, Qwen3-0.6B-shaped ranker, {wl.n_items}-item FP16 table",
+        "requests_per_gpu": len(wl.requests),
+        "candidates_per_gpu": wl.n_candidates,
+        "tokens_per_gpu": wl.n_tokens,
+        "prefix_len_mean": round(float(np.mean(Ls)), 1),
+        "mode": mode,
+        "cuda_graph": graph,
+        "parallelism": f"dp{n}",
+        "weights": "bf16 values, stored exactly as fp16 x 2^s",
+        "l2": "no flush: the step's working set (0.88 GB weights + activations) exceeds the 126 MB L2",
+    }
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work per step
+# ---------------------------------------------------------------------------
+
+def gemm_flops(shape: W.ModelShape, T: int) -> float:
+    d, qd, kd, F = shape.d, shape.q_dim, shape.kv_dim, shape.ffn
+    return 2.0 * T * (d * (qd + 2 * kd) + qd * d + d * 2 * F + F * d) * shape.n_layers
+
+
+def attention_pairs(wl: W.Workload, independent: bool) -> int:
+    b = wl.branch_len
+    tot = 0
+    for r in wl.requests:
+        L, K = r.L, r.K
+        if independent:
+            tot += K * (L + b) * (L + b + 1) // 2
+        else:
+            tot += L * (L + 1) // 2 + K * sum(L + i + 1 for i in range(b))
+    return tot
+
+
+def attention_flops(shape: W.ModelShape, wl: W.Workload, independent: bool) -> float:
+    # QK^T and PV: 2 * head_dim each per (query, key) pair and query head
+    return 4.0 * shape.head_dim * shape.n_q_heads * attention_pairs(wl, independent) * shape.n_layers
+
+
+def attention_bytes(shape: W.ModelShape, T: int) -> float:
+    # q read, k and v read once, o written (fp16), per layer
+    return 2.0 * T * (2 * shape.q_dim + 2 * shape.kv_dim) * shape.n_layers
+
+
+def peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            m = json.load(f)
+        return {"hbm": m["hbm_gbs"], "tc": m["bf16_tflops"], "tc_sustained": m["bf16_tflops_sustained"],
+                "src": "measured"}
+    return {"hbm": 6650.0, "tc": 1590.0, "tc_sustained": 1400.0, "src": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([c.strip() for c in line.split(",")])
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            try:
+                sm.append(float(r[0]))
+                mx = float(r[1])
+                for n, v in zip(names, r[3:7]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        loaded = [v for v in sm if v > 0.5 * (mx or max(sm))] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing
+# ---------------------------------------------------------------------------
+
+def oracle_time(wl: W.Workload, requests, warmup: int = 1) -> tuple:
+    """Score the given requests with the oracle; returns (seconds per request,
+    candidates).  `warmup` short calls first load the library and page in the
+    weights."""
+    from oracle import ranker as R
+    om = R.OracleModel(wl.model, W.model_weights(wl.model))
+    rho = R.embedding_rho(om.embed)
+    a = W.item_vectors(wl.n_items, wl.model.d)
+    rows = set()
+    for q in requests:
+        r = wl.requests[q]
+        for i in np.concatenate([r.prefix_ids, r.branch_ids.reshape(-1)]):
+            if i >= wl.model.vocab:
+                rows.add(int(i) - wl.model.vocab)
+    rows = np.array(sorted(rows), np.int64)
+    sub = R.table_f32(R.interface(a[rows], 0.0, rho))
+    remap = {int(r): i for i, r in enumerate(rows)}
+
+    def rm(ids):
+        return np.array([i if i < wl.model.vocab else wl.model.vocab + remap[int(i) - wl.model.vocab]
+                         for i in ids.reshape(-1)], np.int32).reshape(ids.shape)
+
+    local = [W.Request(rm(wl.requests[q].prefix_ids), rm(wl.requests[q].branch_ids)) for q in requests]
+    for _ in range(max(1, warmup)):
+        R.score_mis(om, sub, W.Request(local[0].prefix_ids[:4], local[0].branch_ids[:1]))
+    per = []
+    n = 0
+    for req in local:
+        t = time.perf_counter()
+        R.score_mis(om, sub, req)
+        per.append(time.perf_counter() - t)
+        n += req.K
+    return per, n
+
+
+def cpu_count() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------------------
+
+def run_reference(args, rank: int, world: int) -> None:
+    if rank != 0:
+        return
+    wl = workload(args.config, 0)
+    steps, warm = args.steps, args.warmup
+    n_req = len(wl.requests)
+    order = [i % n_req for i in range(steps)]
+    per, _ = oracle_time(wl, order, warmup=warm)
+    cands = sum(wl.requests[q].K for q in order)
+    total = sum(per)
+    value = cands / total
+    sample = (f"{steps} timed steps, step i = request i of the {wl.name} batch (all its candidates) scored by "
+              f"the oracle's packed layout; {warm} warm-up calls on a 4-token slice of request 0")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps, "warmup": warm,
+        "ms_per_step": 1e3 * total / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": describe(wl, args.mode, False, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_count(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank: int, world: int, local_rank: int) -> None:
+    import torch
+
+    import shared_prefix_item_b200 as S
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+
+    wl = workload(args.config, rank)
+    shape = wl.model
+    mode = S.MODE_INDEPENDENT if args.mode == "independent" else S.MODE_MIS
+    # the library launches on this stream; the CUDA events below are recorded on it
+    stream = torch.cuda.Stream()
+    torch.cuda.set_stream(stream)
+    rk = S.Ranker(shape, W.model_weights(shape), device=local_rank, stream=stream.cuda_stream)
+    rk.vid_table_build(W.item_vectors(wl.n_items, shape.d), 0.0, rk.embedding_rho())
+    rk.set_graph(not args.no_graph)
+    p, po, b, co = wl.packed()
+    rk.prepare(p, po, b, co, wl.branch_len, mode)
+    n_cand = wl.n_candidates
+    T = int(rk.debug_layout()[0].shape[0])
+
+    if args.profile_steps:
+        # a short run for ncu captures: N passes kernel by kernel, no timing
+        rk.set_graph(False)
+        for _ in range(args.profile_steps):
+            rk.execute()
+        rk.sync()
+        rk.close()
+        return
+
+    for _ in range(args.warmup):
+        rk.execute()
+    rk.sync()
+
+    def barrier():
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    props = torch.cuda.get_device_properties(local_rank)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local_rank)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_id) as clk:
+        barrier()
+        start.record(stream)
+        for _ in range(args.steps):
+            rk.execute()
+        end.record(stream)
+        barrier()
+    rk.sync()
+    ms = start.elapsed_time(end) / args.steps
+    ms_t = torch.tensor([ms], device="cuda")
+    if dist:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    value = n_cand * world / (ms_max / 1e3)
+    launches = rk.launches_per_execute()
+
+    # e2e: the public call from host buffers, scores back to the host every step
+    out = np.empty(n_cand, np.float32)
+    rk.score(p, po, b, co, wl.branch_len, mode, out=out)
+    h2d = rk.plan_bytes()
+    barrier()
+    start.record(stream)
+    for _ in range(args.steps):
+        rk.score(p, po, b, co, wl.branch_len, mode, out=out)
+    end.record(stream)
+    barrier()
+    e2e_ms = start.elapsed_time(end) / args.steps
+    e2e_t = torch.tensor([e2e_ms], device="cuda")
+    if dist:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+    e2e_value = n_cand * world / (float(e2e_t.item()) / 1e3)
+
+    # per-kernel-class device time (eager launches with an event after each)
+    rk.prepare(p, po, b, co, wl.branch_len, mode)
+    prof = rk.profile(max(2, min(args.steps, 5)))
+    steps_prof = max(2, min(args.steps, 5))
+    pk = peaks()
+    indep = mode == S.MODE_INDEPENDENT
+    g_ms = sum(prof[k][0] for k in ("gemm_qkv", "gemm_o", "gemm_gate_up", "gemm_down")) / steps_prof
+    g_n = sum(prof[k][1] for k in ("gemm_qkv", "gemm_o", "gemm_gate_up", "gemm_down")) / steps_prof
+    a_ms = prof["attention"][0] / steps_prof
+    a_n = prof["attention"][1] / steps_prof
+    gf = gemm_flops(shape, T)
+    af = attention_flops(shape, wl, indep)
+    kernels = {k: {"ms_per_step": round(v[0] / steps_prof, 4), "launches_per_step": v[1] // steps_prof}
+               for k, v in prof.items()}
+    tot_ms = sum(v["ms_per_step"] for v in kernels.values())
+    for v in kernels.values():
+        v["share"] = round(v["ms_per_step"] / tot_ms, 4) if tot_ms else None
+    gemm_roof = {"bound": "tensor", "achieved": gf / (g_ms / 1e3) / 1e12, "peak": pk["tc_sustained"],
+                 "unit": "TFLOP/s", "kernel": "gemm_tc_kernel (QKV, O, gate/up, down)",
+                 "launches_per_step": g_n, "flops_per_launch": gf / max(g_n, 1)}
+    attn_roof = {"bound": "tensor", "achieved": af / (a_ms / 1e3) / 1e12, "peak": pk["tc_sustained"],
+                 "unit": "TFLOP/s", "kernel": "attention_f16_kernel",
+                 "launches_per_step": a_n, "flops_per_launch": af / max(a_n, 1),
+                 "hbm_gbs_algorithmic": attention_bytes(shape, T) / (a_ms / 1e3) / 1e9}
+    for r in (gemm_roof, attn_roof):
+        r["frac"] = r["achieved"] / r["peak"]
+        r["peak_note"] = f"{pk['src']} sustained bf16 dense (fp16 runs at the bf16 rate)"
+        r["traffic"] = None
+    dominant = gemm_roof if g_ms >= a_ms else attn_roof
+    step_roof_ms = max((gf + af) / (pk["tc_sustained"] * 1e12), 0.0) * 1e3
+    cpu = None
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        per, nc = oracle_time(wl, [0])
+        cpu = {"value": nc / sum(per), "unit": UNIT, "cores": cpu_count(), "kind": "oracle",
+               "sample": f"request 0 of the {wl.name} batch (L={wl.requests[0].L}, K={wl.requests[0].K}) "
+                         f"through the oracle's packed layout, {sum(per):.1f} s"}
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": value / H100_C64 if args.config == "c64" and not indep else None,
+            "dtype": "f16", "data": "synthetic",
+            "config": describe(wl, args.mode, not args.no_graph, world),
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4 * n_cand},
+            "roofline": dominant,
+            "roofline_step": {"flops_per_step": gf + af, "ms_at_peak": step_roof_ms,
+                              "frac": step_roof_ms / ms_max, "peak": pk["tc_sustained"],
+                              "unit": "TFLOP/s", "note": "whole step vs max(FLOPs/peak, bytes/HBM BW)"},
+            "roofline_other": attn_roof if dominant is gemm_roof else gemm_roof,
+            "kernels": kernels,
+            "gpu_launches": launches * args.steps,
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    rk.close()
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="c64")
+    ap.add_argument("--mode", choices=["mis", "independent"], default="mis")
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--profile-steps", type=int, default=0,
+                    help="only run this many passes kernel by kernel (for ncu), print nothing")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        print(f"note: --warmup {args.warmup} is below the 3 warm-up steps a reported number needs",
+              file=sys.stderr)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

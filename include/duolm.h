@@ -203,6 +203,15 @@ int64_t duolm_plan_bytes(const duolm_ctx *ctx);
  */
 int duolm_debug_gemm(duolm_ctx *ctx, int layer, int which, const uint16_t *a, float *out);
 
+/*
+ * Failure-detection self test: launch one kernel that waits on an mbarrier
+ * nothing ever arrives on, through the same bounded wait the GEMM kernels
+ * use.  The wait gives up after its time limit (2 s), records
+ * "wait-timeout" in the device status word and returns; the call then
+ * returns DUOLM_E_DEVICE and the context stays usable.
+ */
+int duolm_debug_wait_timeout(duolm_ctx *ctx);
+
 /* Kernel classes of duolm_profile. */
 #define DUOLM_PROF_EMBED 0
 #define DUOLM_PROF_GEMM_QKV 1

@@ -65,6 +65,7 @@ def _load():
         "duolm_plan_bytes": (I64, [VP]),
         "duolm_debug_gemm": (I, [VP, I, I, VP, VP]),
         "duolm_profile": (I, [VP, I, VP, VP]),
+        "duolm_debug_wait_timeout": (I, [VP]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -220,6 +221,9 @@ class Ranker:
         out = np.empty((a.shape[0], n_out), np.float32)
         self._check(lib.duolm_debug_gemm(self.ctx, int(layer), int(which), _p(a), _p(out)))
         return out
+
+    def debug_wait_timeout(self):
+        self._check(lib.duolm_debug_wait_timeout(self.ctx))
 
     def debug_table(self, n_items: int) -> np.ndarray:
         out = np.empty((n_items, self.d), np.uint16)

@@ -397,6 +397,24 @@ cudaError_t embed_rho(const void* embed, bool embed_bf16, int64_t vocab, int d, 
   return cudaGetLastError();
 }
 
+// A wait that nothing completes: exercises the bounded-wait error path.
+__global__ void wait_timeout_kernel(DevStatus* st) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t a = smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(a, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(a, 0, st, 90);
+  __syncthreads();
+}
+
+cudaError_t debug_wait_timeout(DevStatus* st, cudaStream_t s) {
+  wait_timeout_kernel<<<1, 32, 0, s>>>(st);
+  return cudaGetLastError();
+}
+
 // The attention kernels' visibility rule evaluated for every pair of one request.
 __global__ void debug_mask_kernel(const PlanHdr* __restrict__ plan, int request, uint8_t* __restrict__ out,
                                   int64_t tq_n) {

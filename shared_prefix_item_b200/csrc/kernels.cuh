@@ -64,6 +64,7 @@ cudaError_t swiglu_f32(const PlanHdr* plan, const float* gu, int F, float* h, in
 cudaError_t table_build(const float* a, int64_t n, int d, double scale_num, __half* out, cudaStream_t s);
 cudaError_t embed_rho(const void* embed, bool embed_bf16, int64_t vocab, int d, double* row_rms, double* out,
                       cudaStream_t s);
+cudaError_t debug_wait_timeout(DevStatus* st, cudaStream_t s);
 cudaError_t debug_mask(const PlanHdr* plan, int request, uint8_t* out, int64_t tq, cudaStream_t s);
 
 // ---- attention

@@ -942,6 +942,13 @@ int duolm_debug_gemm(duolm_ctx* ctx, int layer, int which, const uint16_t* a, fl
   return check_status(ctx);
 }
 
+int duolm_debug_wait_timeout(duolm_ctx* ctx) {
+  if (!ctx) return DUOLM_E_ARG;
+  CK(cudaSetDevice(ctx->device));
+  CK(debug_wait_timeout(ctx->status, ctx->stream));
+  return duolm_sync(ctx);
+}
+
 int duolm_profile(duolm_ctx* ctx, int n_steps, double* ms_out, int64_t* count_out) {
   if (!ctx || !ms_out || !count_out || n_steps < 1) return fail(ctx, DUOLM_E_ARG, "profile: bad arguments");
   if (!ctx->prepared) return fail(ctx, DUOLM_E_STATE, "profile: nothing prepared");

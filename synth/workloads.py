@@ -218,20 +218,21 @@ def tiny(seed_offset: int = 0) -> Workload:
     return Workload("tiny", m, 64, 1, [r])
 
 
-def c1() -> Workload:
+def c1(shard: int = 0) -> Workload:
     """Qwen3-0.6B shape, one request: L = 32 + 10 x (2 + 24) + 4 = 296, K = 100, b = 1."""
     m = QWEN3_06B
-    s = Stream(SEED_REQUESTS + 1, 0)
+    s = Stream(SEED_REQUESTS + 1, shard)
     tpl = _Template(s, m.vocab, 32, 4, 0)
     r = make_request(s, tpl, m.vocab, 100_000, 10, [24] * 10, 100, 1)
     return Workload("c1", m, 100_000, 1, [r])
 
 
-def c64(n_requests: int = 64) -> Workload:
+def c64(n_requests: int = 64, shard: int = 0) -> Workload:
     """Qwen3-0.6B shape, 64 ragged requests: history U{1..20} items, feedback
-    U{8..48} tokens per item, K = 100, items uniform over 100k."""
+    U{8..48} tokens per item, K = 100, items uniform over 100k.  ``shard``
+    selects an independent batch of the same recipe (one per GPU)."""
     m = QWEN3_06B
-    s = Stream(SEED_REQUESTS + 2, 0)
+    s = Stream(SEED_REQUESTS + 2, shard)
     tpl = _Template(s, m.vocab, 32, 4, 0)
     reqs = []
     for _ in range(n_requests):
@@ -241,22 +242,22 @@ def c64(n_requests: int = 64) -> Workload:
     return Workload("c64", m, 100_000, 1, reqs)
 
 
-def stress(n_requests: int = 16) -> Workload:
+def stress(n_requests: int = 16, shard: int = 0) -> Workload:
     """Long history: 16 requests, L = 32 + 50 x (2 + 40) = 2132, K = 256,
     b = 4 (3 fixed header tokens + the candidate VID)."""
     m = QWEN3_06B
-    s = Stream(SEED_REQUESTS + 3, 0)
+    s = Stream(SEED_REQUESTS + 3, shard)
     tpl = _Template(s, m.vocab, 32, 0, 3)
     reqs = [make_request(s, tpl, m.vocab, 100_000, 50, [40] * 50, 256, 4) for _ in range(n_requests)]
     return Workload("stress", m, 100_000, 4, reqs)
 
 
-def catalog(concurrency: int) -> Workload:
+def catalog(concurrency: int, shard: int = 0) -> Workload:
     """1M-item table, Zipf(1.1) item ids, history 10 x 24 feedback tokens,
     K = 100, header 4; concurrency C in {1, 8, 64}."""
     m = QWEN3_06B
     n_items = 1_000_000
-    s = Stream(SEED_REQUESTS + 4, concurrency)
+    s = Stream(SEED_REQUESTS + 4, concurrency + 1000 * shard)
     tpl = _Template(s, m.vocab, 32, 4, 0)
     draw = _zipf_sampler(n_items, 1.1)
     reqs = [make_request(s, tpl, m.vocab, n_items, 10, [24] * 10, 100, 1, item_draw=draw)
