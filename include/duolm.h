@@ -170,6 +170,41 @@ const char *duolm_last_error(const duolm_ctx *ctx);
 /* Free every device resource of the context (NULL is ignored). */
 void duolm_destroy(duolm_ctx *ctx);
 
+/* Largest vocabulary duolm_embedding_rho_static accepts (rows of its
+ * built-in scratch array: 2 MB of fp64, held by every GPU that loads the
+ * library until the process exits). */
+#define DUOLM_RHO_STATIC_MAX_ROWS 262144
+
+/*
+ * duolm_embedding_rho_static -- the reference scale rho of duolm_embedding_rho
+ * (mean over embedding rows of each row's RMS, fp64) for callers that must
+ * not allocate device memory.  The paper has no counterpart: it is a
+ * deployment aid.  Some callers cannot call cudaMalloc: a serving process
+ * that has already carved all of the GPU's memory into its own pools gets an
+ * out-of-memory failure or a fragmented pool from a fresh allocation, and a
+ * latency-critical loop cannot afford an allocation that may wait for the
+ * whole device.  This entry point allocates nothing: its per-row scratch is a
+ * fixed array of DUOLM_RHO_STATIC_MAX_ROWS doubles built into the library.
+ *   embed:  device pointer to the embedding, [vocab][d] row-major, uint16
+ *           bfloat16 bit patterns (dtype DUOLM_DTYPE_BF16) or float
+ *           (DUOLM_DTYPE_FP32); read only.
+ *   rho_out: device pointer to one double; written by the call.
+ *   cuda_stream: the cudaStream_t to launch on (NULL: the default stream).
+ * The call only enqueues work on the stream of the current device and
+ * returns; rho_out is valid once that stream has reached it.  The first call
+ * on each device looks up the scratch array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture.  Every element of the scratch a call reads is first written by
+ * the same call, so nothing needs clearing, but all calls in the process
+ * share the one array: calls whose work overlaps on the GPU (different
+ * streams, no ordering between them) race and may return wrong results.
+ * Returns 0; DUOLM_E_ARG for a null pointer, d < 1 or a bad dtype;
+ * DUOLM_E_CAPACITY when vocab is < 1 or above DUOLM_RHO_STATIC_MAX_ROWS;
+ * DUOLM_E_CUDA when the address lookup or a launch fails.
+ */
+int duolm_embedding_rho_static(const void *embed, int dtype, int64_t vocab, int d, double *rho_out,
+                               void *cuda_stream);
+
 /* ---- introspection (tests) --------------------------------------------- */
 
 /* Packed layout of the prepared batch as the device holds it: n_tokens,

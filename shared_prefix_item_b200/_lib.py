@@ -66,6 +66,7 @@ def _load():
         "duolm_debug_gemm": (I, [VP, I, I, VP, VP]),
         "duolm_profile": (I, [VP, I, VP, VP]),
         "duolm_debug_wait_timeout": (I, [VP]),
+        "duolm_embedding_rho_static": (I, [VP, I, I64, I, VP, VP]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -75,6 +76,18 @@ def _load():
 
 
 lib = _load()
+
+
+RHO_STATIC_MAX_ROWS = 262144
+
+
+def embedding_rho_static(embed_dev: int, dtype: int, vocab: int, d: int, rho_out_dev: int,
+                         stream: Optional[int] = None) -> None:
+    """duolm_embedding_rho_static: device pointers in, nothing allocated."""
+    rc = lib.duolm_embedding_rho_static(ctypes.c_void_p(embed_dev), int(dtype), int(vocab), int(d),
+                                        ctypes.c_void_p(rho_out_dev), ctypes.c_void_p(stream or 0))
+    if rc != 0:
+        raise DuolmError(rc, f"duolm_embedding_rho_static(vocab={vocab}, d={d}, dtype={dtype}) failed")
 
 
 def _arr(a, dtype) -> np.ndarray:
