@@ -112,8 +112,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 #pragma unroll
     for (int j = 0; j < 16; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
     const int slot_a = warp * 16 + (lane >> 2);
-    const int tq_a = q0 + slot_a / G;
-    const int tq_b = q0 + (slot_a + 8) / G;
+    const KeyRange kr_a = tree_keys(q0 + slot_a / G, L, b);
+    const KeyRange kr_b = tree_keys(q0 + (slot_a + 8) / G, L, b);
 
     uint32_t qf[8][4];
     for (int t = 0; t < n_tiles; ++t) {
@@ -155,8 +155,12 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         }
       }
 
-      // mask: keys beyond the prefix in the prefix loop of a branch item, and
-      // the tree rule wherever a tile can reach the item's own rows
+      // tree mask on the tiles that can reach keys a row may not see: the
+      // causal diagonal of prefix items, the prefix end and the branch tile
+      // of branch items
+      // The visible keys of a row are [0, pre_hi] in the prefix and
+      // [br_lo, br_hi] in its own branch; prefix tiles take the first part,
+      // the branch tile the second (the two never overlap: br_lo >= L).
       const bool is_branch_tile = branch && t == n_prefix_tiles;
       const bool need_mask = is_branch_tile || (!branch && k0 + kKT > row0) || (branch && k0 + kKT > L);
       float tmax[2] = {-INFINITY, -INFINITY};
@@ -166,15 +170,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         for (int e = 0; e < 4; ++e) {
           float v = s[j][e] * scale_log2;
           if (need_mask) {
+            const KeyRange& kr = e < 2 ? kr_a : kr_b;
             const int tk = k0 + j * 8 + 2 * (lane & 3) + (e & 1);
-            const int tq = (e < 2) ? tq_a : tq_b;
-            bool vis;
-            if (is_branch_tile)
-              vis = tree_visible(tq, tk, L, b);
-            else if (branch)
-              vis = tk < L;
-            else
-              vis = tree_visible(tq, tk, L, b);
+            const bool vis = is_branch_tile ? (tk >= kr.br_lo && tk <= kr.br_hi) : (tk <= kr.pre_hi);
             if (!vis) v = -INFINITY;
           }
           s[j][e] = v;
@@ -188,7 +186,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         tmax[h] = fmaxf(tmax[h], __shfl_xor_sync(0xffffffffu, tmax[h], 2));
         const float m_new = fmaxf(m_run[h], tmax[h]);
         const float m_use = m_new == -INFINITY ? 0.f : m_new;
-        corr[h] = exp2f(m_run[h] - m_use);
+        corr[h] = fast_exp2(m_run[h] - m_use);
         m_run[h] = m_new;
         tmax[h] = m_use;
         l_run[h] *= corr[h];
@@ -198,7 +196,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       for (int j = 0; j < 8; ++j) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float p = exp2f(s[j][e] - tmax[e >> 1]);
+          const float p = fast_exp2(s[j][e] - tmax[e >> 1]);
           s[j][e] = p;
           psum[e >> 1] += p;
         }

@@ -280,12 +280,13 @@ __global__ void qkv_post_f32_kernel(const PlanHdr* __restrict__ plan, const floa
       raise_error(st, ERR_BAD_INDEX, 32);
       p = 0;
     }
-    const float2* cs = rope + (int64_t)p * half;
+    const float2* cs = rope + p;  // entry (i, p) at cs[i * max_pos]
     for (int i = 0; i < half; ++i) {
       const float a = (src[i] * r) * g[i];
       const float bb = (src[i + half] * r) * g[i + half];
-      dst[i] = a * cs[i].x - bb * cs[i].y;
-      dst[i + half] = bb * cs[i].x + a * cs[i].y;
+      const float2 t = cs[(int64_t)i * max_pos];
+      dst[i] = a * t.x - bb * t.y;
+      dst[i + half] = bb * t.x + a * t.y;
     }
   }
 }

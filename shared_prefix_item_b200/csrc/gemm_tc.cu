@@ -1,13 +1,15 @@
 // Projection GEMMs of the ranker on 5th-generation tensor cores (sm_100a).
 //
 // C[M, N] = A[M, K] * B[N, K]^T with fp16 operands and fp32 accumulation in
-// tensor memory.  One persistent CTA per SM, 192 threads, warp-specialised:
+// tensor memory.  One persistent CTA per SM, warp-specialised:
 //   warp 0      TMA producer: streams 128x64 A and BNx64 B tiles (128-byte
 //               swizzle, no multicast) into a STAGES-deep shared-memory ring;
 //   warp 1      allocates 2*BN TMEM columns; lane 0 issues tcgen05.mma
 //               (128 x BN x 16 per instruction) and commits to mbarriers;
-//   warps 2-5   epilogue: each thread owns one accumulator row (TMEM lane),
-//               reads it with tcgen05.ld and applies a fused epilogue.
+//   warps 2..   epilogue, in groups of four warps (one per TMEM lane
+//               quadrant): each thread owns one accumulator row and its
+//               group's share of the columns, reads them with tcgen05.ld and
+//               applies a fused epilogue.
 // Two accumulator buffers let the epilogue of tile i overlap the mainloop of
 // tile i+1.  Every mbarrier wait is bounded (see common.cuh).
 #include <cstdio>
@@ -19,7 +21,6 @@ namespace duolm {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;  // one 128-byte swizzle row of fp16
-constexpr int kThreads = 192;
 
 template <int BN>
 struct TcCfg {
@@ -34,27 +35,38 @@ struct TcCfg {
 };
 
 // ---------------------------------------------------------------------------
-// fused epilogues.  `taddr` addresses this thread's row, column 0 of the tile's
-// accumulator; all lanes of the warp must execute the TMEM loads.
+// fused epilogues.  EG groups of four warps share each tile: group g handles
+// columns [g * BN / EG, (g + 1) * BN / EG) (for QKV, head g of the tile).
+// `taddr` addresses this thread's row, column 0 of the tile's accumulator;
+// all lanes of a warp execute the TMEM loads.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ float silu_fast(float g) {
+  return __fdividef(g, 1.0f + fast_exp2(-1.4426950408889634f * g));
+}
+
 struct EpiResid {
   EpiResidArgs a;
+  static constexpr int EG = 4;
   template <int BN>
-  __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, bool row_ok, const PlanHdr*, DevStatus*) const {
+  __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, int g, bool row_ok, const PlanHdr*,
+                                      DevStatus*) const {
+    constexpr int W = BN / EG;
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = g * W; c < (g + 1) * W; c += 32) {
       float v[32];
       tmem_ld32(taddr + c, v);
       if (row_ok) {
         float4* p = reinterpret_cast<float4*>(a.x + (int64_t)row * a.ldx + n0 + c);
+        float4 t[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) t[j] = p[j];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          float4 t = p[j];
-          t.x += v[4 * j + 0] * a.scale;
-          t.y += v[4 * j + 1] * a.scale;
-          t.z += v[4 * j + 2] * a.scale;
-          t.w += v[4 * j + 3] * a.scale;
-          p[j] = t;
+          t[j].x += v[4 * j + 0] * a.scale;
+          t[j].y += v[4 * j + 1] * a.scale;
+          t[j].z += v[4 * j + 2] * a.scale;
+          t[j].w += v[4 * j + 3] * a.scale;
+          p[j] = t[j];
         }
       }
     }
@@ -63,22 +75,24 @@ struct EpiResid {
 
 struct EpiSwiglu {
   EpiSwigluArgs a;
+  static constexpr int EG = 4;
   template <int BN>
-  __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, bool row_ok, const PlanHdr*,
+  __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, int g, bool row_ok, const PlanHdr*,
                                       DevStatus* st) const {
-    constexpr int H = BN / 2;
+    constexpr int H = BN / 2;   // gate columns [0, H), up columns [H, BN)
+    constexpr int W = H / EG;   // outputs of this group
     const int out0 = n0 / 2;
 #pragma unroll 1
-    for (int c = 0; c < H; c += 32) {
-      float g[32], u[32];
-      tmem_ld32(taddr + c, g);
-      tmem_ld32(taddr + H + c, u);
+    for (int c = g * W; c < (g + 1) * W; c += 32) {
+      float gv[32], uv[32];
+      tmem_ld32(taddr + c, gv);
+      tmem_ld32(taddr + H + c, uv);
       if (row_ok) {
         uint32_t packed[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          float h0 = silu(g[2 * j] * a.scale) * (u[2 * j] * a.scale);
-          float h1 = silu(g[2 * j + 1] * a.scale) * (u[2 * j + 1] * a.scale);
+          const float h0 = silu_fast(gv[2 * j] * a.scale) * (uv[2 * j] * a.scale);
+          const float h1 = silu_fast(gv[2 * j + 1] * a.scale) * (uv[2 * j + 1] * a.scale);
           __half2 hh = __halves2half2(to_half_checked(h0, st, 20), to_half_checked(h1, st, 20));
           packed[j] = *reinterpret_cast<uint32_t*>(&hh);
         }
@@ -95,104 +109,106 @@ struct EpiSwiglu {
 // copied.  q goes to [T][Hq][128], k and v to the per-head KV buffers.
 struct EpiQkv {
   EpiQkvArgs a;
+  static constexpr int EG = 2;  // one head of the 256-column tile per group
   template <int BN>
-  __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, bool row_ok, const PlanHdr* plan,
+  __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, int g, bool row_ok, const PlanHdr* plan,
                                       DevStatus* st) const {
-    const int* pos_arr = plan_array<int32_t>(plan, plan->off_pos);
+    const int gc = n0 + 128 * g;
+    const uint32_t base = taddr + 128 * g;
+    if (gc >= a.qd + a.kd) {  // value head
+      const int head = (gc - a.qd - a.kd) >> 7;
+      __half* dst = a.vc + ((int64_t)head * a.kv_rows + row) * 128;
 #pragma unroll 1
-    for (int hl = 0; hl < BN / 128; ++hl) {
-      const int gc = n0 + 128 * hl;
-      const uint32_t base = taddr + 128 * hl;
-      if (gc >= a.qd + a.kd) {  // value head
-        const int head = (gc - a.qd - a.kd) >> 7;
-        __half* dst = a.vc + ((int64_t)head * a.kv_rows + row) * 128;
-#pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
-          float v[32];
-          tmem_ld32(base + c, v);
-          if (row_ok) {
-            uint32_t pk[16];
+      for (int c = 0; c < 128; c += 16) {
+        float v[16];
+        tmem_ld16(base + c, v);
+        if (row_ok) {
+          uint32_t pk[8];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              __half2 hh = __halves2half2(to_half_checked(v[2 * j] * a.scale, st, 21),
-                                          to_half_checked(v[2 * j + 1] * a.scale, st, 21));
-              pk[j] = *reinterpret_cast<uint32_t*>(&hh);
-            }
-            uint4* p = reinterpret_cast<uint4*>(dst + c);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) p[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          for (int j = 0; j < 8; ++j) {
+            __half2 hh = __halves2half2(to_half_checked(v[2 * j] * a.scale, st, 21),
+                                        to_half_checked(v[2 * j + 1] * a.scale, st, 21));
+            pk[j] = *reinterpret_cast<uint32_t*>(&hh);
           }
+          uint4* p = reinterpret_cast<uint4*>(dst + c);
+          p[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          p[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
-        continue;
       }
-      const bool is_q = gc < a.qd;
-      const int head = is_q ? (gc >> 7) : ((gc - a.qd) >> 7);
-      const float* gain = is_q ? a.gq : a.gk;
-      __half* dst = is_q ? a.q + ((int64_t)row * a.n_q_heads + head) * 128
-                         : a.kc + ((int64_t)head * a.kv_rows + row) * 128;
-      float ss = 0.f;
+      return;
+    }
+    const bool is_q = gc < a.qd;
+    const int head = is_q ? (gc >> 7) : ((gc - a.qd) >> 7);
+    const float* gain = is_q ? a.gq : a.gk;
+    __half* dst = is_q ? a.q + ((int64_t)row * a.n_q_heads + head) * 128
+                       : a.kc + ((int64_t)head * a.kv_rows + row) * 128;
+    float ss = 0.f;
 #pragma unroll 1
-      for (int c = 0; c < 128; c += 32) {
-        float v[32];
-        tmem_ld32(base + c, v);
+    for (int c = 0; c < 128; c += 16) {
+      float v[16];
+      tmem_ld16(base + c, v);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          float t = v[j] * a.scale;
-          ss += t * t;
-        }
+      for (int j = 0; j < 16; ++j) {
+        const float t = v[j] * a.scale;
+        ss += t * t;
       }
-      const float r = rsqrtf(ss * (1.0f / 128.0f) + a.eps);
-      int p = row_ok ? pos_arr[row] : 0;
+    }
+    const float r = rsqrtf(ss * (1.0f / 128.0f) + a.eps);
+    int p = 0;
+    if (row_ok) {
+      p = plan_array<int32_t>(plan, plan->off_pos)[row];
       if (p < 0 || p >= a.max_pos) {
-        if (row_ok) raise_error(st, ERR_BAD_INDEX, 22);
+        raise_error(st, ERR_BAD_INDEX, 22);
         p = 0;
       }
-      const float2* cs = a.rope + (int64_t)p * 64;
+    }
+    const float2* cs = a.rope + p;  // entry (i, p) at cs[i * max_pos]
 #pragma unroll 1
-      for (int c = 0; c < 64; c += 32) {
-        float x1[32], x2[32];
-        tmem_ld32(base + c, x1);
-        tmem_ld32(base + 64 + c, x2);
-        if (row_ok) {
-          uint32_t o1[16], o2[16];
+    for (int c = 0; c < 64; c += 16) {
+      float x1[16], x2[16];
+      tmem_ld16(base + c, x1);
+      tmem_ld16(base + 64 + c, x2);
+      if (row_ok) {
+        uint32_t o1[8], o2[8];
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            float r1[2], r2[2];
+        for (int j = 0; j < 16; j += 2) {
+          float r1[2], r2[2];
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int i = c + j + e;
-              const float a1 = (x1[j + e] * a.scale * r) * gain[i];
-              const float a2 = (x2[j + e] * a.scale * r) * gain[64 + i];
-              const float2 t = cs[i];
-              r1[e] = a1 * t.x - a2 * t.y;
-              r2[e] = a2 * t.x + a1 * t.y;
-            }
-            __half2 h1 = __floats2half2_rn(r1[0], r1[1]);
-            __half2 h2 = __floats2half2_rn(r2[0], r2[1]);
-            o1[j / 2] = *reinterpret_cast<uint32_t*>(&h1);
-            o2[j / 2] = *reinterpret_cast<uint32_t*>(&h2);
+          for (int e = 0; e < 2; ++e) {
+            const int i = c + j + e;
+            const float a1 = (x1[j + e] * a.scale * r) * gain[i];
+            const float a2 = (x2[j + e] * a.scale * r) * gain[64 + i];
+            const float2 t = cs[(int64_t)i * a.max_pos];
+            r1[e] = a1 * t.x - a2 * t.y;
+            r2[e] = a2 * t.x + a1 * t.y;
           }
-          uint4* p1 = reinterpret_cast<uint4*>(dst + c);
-          uint4* p2 = reinterpret_cast<uint4*>(dst + 64 + c);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            p1[j] = make_uint4(o1[4 * j], o1[4 * j + 1], o1[4 * j + 2], o1[4 * j + 3]);
-            p2[j] = make_uint4(o2[4 * j], o2[4 * j + 1], o2[4 * j + 2], o2[4 * j + 3]);
-          }
+          __half2 h1 = __floats2half2_rn(r1[0], r1[1]);
+          __half2 h2 = __floats2half2_rn(r2[0], r2[1]);
+          o1[j / 2] = *reinterpret_cast<uint32_t*>(&h1);
+          o2[j / 2] = *reinterpret_cast<uint32_t*>(&h2);
         }
+        uint4* p1 = reinterpret_cast<uint4*>(dst + c);
+        uint4* p2 = reinterpret_cast<uint4*>(dst + 64 + c);
+        p1[0] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+        p1[1] = make_uint4(o1[4], o1[5], o1[6], o1[7]);
+        p2[0] = make_uint4(o2[0], o2[1], o2[2], o2[3]);
+        p2[1] = make_uint4(o2[4], o2[5], o2[6], o2[7]);
       }
     }
   }
 };
 
 // ---------------------------------------------------------------------------
-// the kernel
+// the kernel: warp 0 TMA producer, warp 1 MMA issuer, warps 2 .. 2 + 4*EG - 1
+// epilogue (group g = (warp - 2) / 4; each group spans the four TMEM lane
+// quadrants, warp w accessing lanes 32 * (w % 4) .. + 31)
 // ---------------------------------------------------------------------------
 template <int BN, class Epi>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(64 + 128 * Epi::EG, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int Kdim,
                    int N, const PlanHdr* __restrict__ plan, const Epi epi, DevStatus* st) {
   using C = TcCfg<BN>;
+  constexpr int EG = Epi::EG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
@@ -220,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull0 + 8 * a, 1);
-      mbar_init(tempty0 + 8 * a, 128);
+      mbar_init(tempty0 + 8 * a, 128 * EG);
     }
     fence_barrier_init();
   }
@@ -292,17 +308,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    const int q4 = warp & 3;  // TMEM lane quadrant this warp may access
+    const int q4 = warp & 3;           // TMEM lane quadrant this warp may access
+    const int group = (warp - 2) >> 2;  // column group of the tile
     int local = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
       const int acc = local & 1;
       const uint32_t use = (uint32_t)(local >> 1);
-      if (!mbar_wait(tfull0 + 8 * acc, use & 1u, st, 4)) break;
+      if (!mbar_wait_warp(tfull0 + 8 * acc, use & 1u, st, 4)) break;
       tc_fence_after();
       const int m_blk = tile % m_tiles, n_blk = tile / m_tiles;
       const int row = m_blk * kBM + q4 * 32 + lane;
       const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q4 * 32) << 16);
-      epi.template run<BN>(taddr, row, n_blk * BN, row < M, plan, st);
+      epi.template run<BN>(taddr, row, n_blk * BN, group, row < M, plan, st);
       tc_fence_before();
       mbar_arrive(tempty0 + 8 * acc);
     }
@@ -355,6 +372,27 @@ bool make_tmap_f16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64
   return true;
 }
 
+bool make_tmap_f16_3d(CUtensorMap* map, const void* base, const uint64_t dims[3], const uint64_t strides_bytes[2],
+                      const uint32_t box[3], char* err, size_t errlen) {
+  PFN_encodeTiled enc = get_encode();
+  if (!enc) {
+    snprintf(err, errlen, "cuTensorMapEncodeTiled unavailable");
+    return false;
+  }
+  cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+  cuuint64_t s[2] = {strides_bytes[0], strides_bytes[1]};
+  cuuint32_t bx[3] = {box[0], box[1], box[2]};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), d, s, bx, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(err, errlen, "cuTensorMapEncodeTiled (3-D) failed (%d)", (int)r);
+    return false;
+  }
+  return true;
+}
+
 int gemm_tc_smem_bytes(int bn) { return bn == 256 ? TcCfg<256>::SMEM : TcCfg<128>::SMEM; }
 
 cudaError_t gemm_tc_setup() {
@@ -371,17 +409,17 @@ cudaError_t gemm_tc_setup() {
 
 cudaError_t gemm_tc_resid(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
                           EpiResidArgs e, DevStatus* st, int grid, cudaStream_t s) {
-  gemm_tc_kernel<256, EpiResid><<<grid, kThreads, TcCfg<256>::SMEM, s>>>(a, b, K, N, plan, EpiResid{e}, st);
+  gemm_tc_kernel<256, EpiResid><<<grid, 64 + 128 * EpiResid::EG, TcCfg<256>::SMEM, s>>>(a, b, K, N, plan, EpiResid{e}, st);
   return cudaGetLastError();
 }
 cudaError_t gemm_tc_swiglu(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
                            EpiSwigluArgs e, DevStatus* st, int grid, cudaStream_t s) {
-  gemm_tc_kernel<256, EpiSwiglu><<<grid, kThreads, TcCfg<256>::SMEM, s>>>(a, b, K, N, plan, EpiSwiglu{e}, st);
+  gemm_tc_kernel<256, EpiSwiglu><<<grid, 64 + 128 * EpiSwiglu::EG, TcCfg<256>::SMEM, s>>>(a, b, K, N, plan, EpiSwiglu{e}, st);
   return cudaGetLastError();
 }
 cudaError_t gemm_tc_qkv(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
                         EpiQkvArgs e, DevStatus* st, int grid, cudaStream_t s) {
-  gemm_tc_kernel<256, EpiQkv><<<grid, kThreads, TcCfg<256>::SMEM, s>>>(a, b, K, N, plan, EpiQkv{e}, st);
+  gemm_tc_kernel<256, EpiQkv><<<grid, 64 + 128 * EpiQkv::EG, TcCfg<256>::SMEM, s>>>(a, b, K, N, plan, EpiQkv{e}, st);
   return cudaGetLastError();
 }
 

@@ -22,7 +22,7 @@ struct EpiQkvArgs {     // per 128-wide head: q/k RMSNorm + RoPE, v copy; fp16 o
   __half* q;            // [T][n_q_heads][128]
   __half* kc;           // [n_kv_heads][kv_rows][128]
   __half* vc;           // [n_kv_heads][kv_rows][128]
-  const float2* rope;   // [max_pos][64] (cos, sin)
+  const float2* rope;   // [64][max_pos] (cos, sin), frequency-major
   int64_t kv_rows;
   int max_pos;
   const float* gq;      // q_norm gains [128]
@@ -34,6 +34,8 @@ struct EpiQkvArgs {     // per 128-wide head: q/k RMSNorm + RoPE, v copy; fp16 o
 
 bool make_tmap_f16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
                       uint32_t box_outer, char* err, size_t errlen);
+bool make_tmap_f16_3d(CUtensorMap* map, const void* base, const uint64_t dims[3], const uint64_t strides_bytes[2],
+                      const uint32_t box[3], char* err, size_t errlen);
 int gemm_tc_smem_bytes(int bn);
 cudaError_t gemm_tc_setup();
 cudaError_t gemm_tc_resid(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
@@ -76,5 +78,11 @@ cudaError_t attention_f32(const PlanHdr* plan, const float* q, const float* kc, 
                           cudaStream_t s);
 int attention_rows_per_item(int group);
 cudaError_t attention_setup();
+// tcgen05 attention (fp16 path): items of 128 query slots, KV tiles of 128 keys
+cudaError_t attention_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const PlanHdr* plan,
+                         int64_t kv_rows, int n_q_heads, int n_kv_heads, float scale, __half* o, DevStatus* st,
+                         int grid, cudaStream_t s);
+cudaError_t attention_tc_setup();
+int attention_tc_rows_per_item(int group);
 
 }  // namespace duolm

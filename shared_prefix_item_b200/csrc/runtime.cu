@@ -24,7 +24,7 @@ using namespace duolm;
 namespace {
 
 constexpr int kMaxPos = 32768;   // position ids must stay below this
-constexpr int kKvPad = 64;       // spare KV rows so a 64-key tile never leaves the buffer
+constexpr int kKvPad = 128;      // spare KV rows so a 128-key tile never leaves the buffer
 constexpr int kPerLayer = 11;
 
 struct LayerW {
@@ -82,6 +82,7 @@ struct duolm_ctx {
   char* plan_host = nullptr;
   cudaEvent_t plan_ev = nullptr;
   CUtensorMap tm_xn, tm_oact, tm_h;
+  CUtensorMap tm_q3, tm_kc, tm_vc;  // attention operands
 
   bool prepared = false;
   int64_t n_tokens = 0, n_cand = 0;
@@ -291,6 +292,14 @@ int reserve_impl(duolm_ctx* ctx, int64_t T, int64_t R, int64_t C) {
         !make_tmap_f16_2d(&ctx->tm_oact, ctx->o, ctx->qd, T, 64, 128, e, sizeof e) ||
         !make_tmap_f16_2d(&ctx->tm_h, ctx->h, d.ffn, T, 64, 128, e, sizeof e))
       return fail(ctx, DUOLM_E_CUDA, "%s", e);
+    // q as [token][head][128]: boxes of 64 dims x (the G heads of one KV head) x (128 / G) tokens
+    const uint64_t qdims[3] = {128, (uint64_t)d.n_q_heads, (uint64_t)T};
+    const uint64_t qstr[2] = {256, (uint64_t)d.n_q_heads * 256};
+    const uint32_t qbox[3] = {64, (uint32_t)ctx->group, (uint32_t)(128 / ctx->group)};
+    if (!make_tmap_f16_3d(&ctx->tm_q3, ctx->q, qdims, qstr, qbox, e, sizeof e) ||
+        !make_tmap_f16_2d(&ctx->tm_kc, ctx->kc, 128, (uint64_t)d.n_kv_heads * kv_rows, 64, 128, e, sizeof e) ||
+        !make_tmap_f16_2d(&ctx->tm_vc, ctx->vc, 128, (uint64_t)d.n_kv_heads * kv_rows, 64, 128, e, sizeof e))
+      return fail(ctx, DUOLM_E_CUDA, "%s", e);
   }
   ctx->prepared = false;
   return 0;
@@ -340,9 +349,8 @@ cudaError_t launch_forward(duolm_ctx* c, int n_layers, bool with_head, int64_t* 
                     kv_rows, kMaxPos, c->gains + L.g_q, c->gains + L.g_k, L.s_qkv, d.rms_eps, c->qd, c->kd,
                     d.n_q_heads};
       LCK(DUOLM_PROF_GEMM_QKV, gemm_tc_qkv(c->tm_xn, L.tm_qkv, d.d, c->qd + 2 * c->kd, plan, qa, c->status, c->num_sms, s));
-      LCK(DUOLM_PROF_ATTENTION, attention_f16(plan, static_cast<__half*>(c->q), static_cast<__half*>(c->kc), static_cast<__half*>(c->vc),
-                        kv_rows, d.n_q_heads, d.n_kv_heads, attn_scale, static_cast<__half*>(c->o), c->status,
-                        2 * c->num_sms, s));
+      LCK(DUOLM_PROF_ATTENTION, attention_tc(c->tm_q3, c->tm_kc, c->tm_vc, plan, kv_rows, d.n_q_heads, d.n_kv_heads,
+                                             attn_scale, static_cast<__half*>(c->o), c->status, c->num_sms, s));
       LCK(DUOLM_PROF_GEMM_O, gemm_tc_resid(c->tm_oact, L.tm_o, c->qd, d.d, plan, EpiResidArgs{c->x, d.d, L.s_o}, c->status,
                         c->num_sms, s));
       LCK(DUOLM_PROF_RMSNORM, rmsnorm_rows<__half>(plan, c->x, d.d, c->gains + L.g_mlp, d.rms_eps, xn, c->status, maxT, s));
@@ -446,7 +454,7 @@ int duolm_model_load(const duolm_model_desc* desc, const void* const* host_weigh
   ctx->qd = d.n_q_heads * d.head_dim;
   ctx->kd = d.n_kv_heads * d.head_dim;
   ctx->group = G;
-  ctx->rows_per_item = ctx->f16 ? attention_rows_per_item(G) : 64;
+  ctx->rows_per_item = ctx->f16 ? attention_tc_rows_per_item(G) : 64;
   auto bail = [&](int rc) {
     g_load_err = ctx->err.empty() ? "model_load failed (code " + std::to_string(rc) + ")" : ctx->err;
     duolm_destroy(ctx);
@@ -532,23 +540,26 @@ int duolm_model_load(const duolm_model_desc* desc, const void* const* host_weigh
       if ((rc = upload_f32(ctx, {P(b + 10, D * F)}, &L.wd))) return bail(rc);
     }
   }
-  // RoPE table: (cos, sin) of pos * theta^(-2i/hd), computed in double
+  // RoPE table: (cos, sin) of pos * theta^(-2i/hd), computed in double,
+  // frequency-major [hd/2][kMaxPos] so that neighbouring tokens read
+  // neighbouring entries
   {
     const int64_t half = hd / 2;
     std::vector<float2> t((size_t)(kMaxPos * half));
-    for (int64_t p = 0; p < kMaxPos; ++p)
-      for (int64_t i = 0; i < half; ++i) {
-        const double inv = std::pow((double)d.rope_theta, -2.0 * (double)i / (double)hd);
+    for (int64_t i = 0; i < half; ++i) {
+      const double inv = std::pow((double)d.rope_theta, -2.0 * (double)i / (double)hd);
+      for (int64_t p = 0; p < kMaxPos; ++p) {
         const double a = (double)p * inv;
-        t[p * half + i] = make_float2((float)std::cos(a), (float)std::sin(a));
+        t[i * kMaxPos + p] = make_float2((float)std::cos(a), (float)std::sin(a));
       }
+    }
     if ((rc = dalloc(ctx, &ctx->rope, t.size() * sizeof(float2)))) return bail(rc);
     if (cudaMemcpy(ctx->rope, t.data(), t.size() * sizeof(float2), cudaMemcpyHostToDevice) != cudaSuccess)
       return bail(DUOLM_E_CUDA);
   }
   if ((rc = dalloc(ctx, &ctx->status, sizeof(DevStatus)))) return bail(rc);
   if (cudaMemset(ctx->status, 0, sizeof(DevStatus)) != cudaSuccess) return bail(DUOLM_E_CUDA);
-  if (ctx->f16 && (gemm_tc_setup() != cudaSuccess || attention_setup() != cudaSuccess)) return bail(DUOLM_E_CUDA);
+  if (ctx->f16 && (gemm_tc_setup() != cudaSuccess || attention_tc_setup() != cudaSuccess)) return bail(DUOLM_E_CUDA);
   *out = ctx;
   return 0;
 }

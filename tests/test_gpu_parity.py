@@ -132,7 +132,8 @@ def test_q2_layout_mask_gather_bit_exact():
     (314, 2, 2, 28, 33, 1, 1),          # L = 63: prefix one short of a key tile
     (315, 1, 1, 60, 64, 1, 0),          # L = 64 exactly, branch rows span 2 items
     (316, 2, 3, (40, 45), (30, 70), 2, 5),  # L > 128: several key tiles, ragged tail
-    (317, 1, 1, 60, 9, 32, 2),          # b = 32: the longest branch the kernel takes
+    (317, 1, 1, 60, 9, 32, 2),          # b = 32: half an attention item
+    (318, 1, 1, 70, 3, 64, 2),          # b = 64: the longest branch the kernel takes
 ])
 def test_q2_ragged_scores(seed, n_req, n_hist, fb, K, b, n_instr):
     wl = W.custom(Q2, Q2_ITEMS, seed, n_req, n_hist, fb, K, b, n_instr=n_instr, n_header=2)
@@ -181,7 +182,7 @@ def test_host_validation_errors():
         rk.score(p, np.array([1, 5, len(p)]), b, co, 1)
     assert e.value.code == -3
     with pytest.raises(S.DuolmError) as e:
-        rk.score(p, po, np.zeros(8 * 33, np.int32), co, 33)  # branch longer than an item
+        rk.score(p, po, np.zeros(8 * 65, np.int32), co, 65)  # branch longer than an item
     assert e.value.code == -1
     # the context is still usable
     ref = rk.score_workload(wl)
