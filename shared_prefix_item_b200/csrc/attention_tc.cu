@@ -10,20 +10,23 @@
 //   kind 1  branch tokens [row0, row0 + R') (whole candidates): every prefix
 //           key, then one extra 128-key tile of branch rows under the tree rule.
 // Per item each KV head's prefix tiles stream through shared memory once for
-// all 128 slots.  One CTA per SM, 192 threads:
-//   warp 0   TMA: Q (3-D map, 2 x 16 KB), then K and V tiles of 128 keys
-//            (2 x 32 KB each, double buffered); 128-byte swizzle, no multicast;
+// all 128 slots.  One CTA per SM, 320 threads:
+//   warp 0   TMA: Q (3-D map, 2 x 16 KB, double buffered so the next item's
+//            Q arrives early), then K and V tiles of 128 keys (2 x 32 KB
+//            each, double buffered); 128-byte swizzle, no multicast;
 //   warp 1   one lane issues tcgen05.mma: S = Q K^T (M 128, N 128 keys,
 //            K-major operands) into one of two TMEM S buffers, then
 //            O += P V (P from shared memory K-major, V MN-major) into TMEM;
 //            S of tile t + 1 is issued before P V of tile t;
-//   warps 2-5 softmax, one thread per slot row (TMEM lane): load S, mask,
-//            row max, P = 2^(s - m) in fp16 to shared memory, row sum; O in
+//   warps 2-9 softmax, two threads per slot row (TMEM lane), each on half of
+//            the keys: load S, mask, row max (halves combined through shared
+//            memory), P = 2^(s - m) in fp16 to shared memory, row sum; O in
 //            TMEM is rescaled only when the running max grows by more than
 //            2^8 (P stays below 256, exact after the final division);
 //            finally O / l to global memory.
-// Every mbarrier wait is bounded; after a timeout the kernel raises the
-// status flag and returns.
+// The three roles run ahead of each other across item boundaries; every
+// mbarrier wait is bounded, and after a timeout the kernel raises the status
+// flag and returns.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -34,21 +37,23 @@ namespace {
 constexpr int kSlots = 128;   // query slots per item (MMA M)
 constexpr int kKeys = 128;    // keys per tile (MMA N of Q K^T)
 constexpr int kHD = 128;
-constexpr int kThreads = 192;
+constexpr int kSoftmax = 256;             // 8 softmax warps: two per TMEM lane quadrant
+constexpr int kThreads = 64 + kSoftmax;
 constexpr int kHalf = 16384;  // one 128-row x 64-element fp16 box
-constexpr int kQOff = 0;                  // Q: 2 boxes
-constexpr int kKOff = 2 * kHalf;          // K: 2 slots x 2 boxes
+constexpr int kQOff = 0;                  // Q: 2 slots x 2 boxes (next item's Q loads early)
+constexpr int kKOff = 4 * kHalf;          // K: 2 slots x 2 boxes
 constexpr int kVOff = kKOff + 4 * kHalf;  // V: 2 slots x 2 boxes
 constexpr int kPOff = kVOff + 4 * kHalf;  // P: 2 boxes
 constexpr int kBarOff = kPOff + 2 * kHalf;
-constexpr int kSmem = kBarOff + 256 + 1024;
+constexpr int kRedOff = kBarOff + 256;     // per-row partial maxima / sums of the two column halves
+constexpr int kSmem = kRedOff + 2 * 128 * 4 + 1024;
 constexpr uint32_t kIdescS = idesc_f16_f32(128, kKeys);
 constexpr uint32_t kIdescPV = idesc_f16_f32_bmn(128, kHD);
 constexpr uint32_t kTmemCols = 512;  // S0 [0,128), S1 [128,256), O [256,384)
 constexpr float kRescaleLog2 = 8.0f;
 
-enum { B_QFULL, B_KVFULL0, B_KVFULL1, B_KVEMPTY0, B_KVEMPTY1, B_SFULL0, B_SFULL1, B_SEMPTY0, B_SEMPTY1,
-       B_PFULL, B_PEMPTY, B_OFULL, B_COUNT };
+enum { B_QFULL0, B_QFULL1, B_QEMPTY0, B_QEMPTY1, B_KVFULL0, B_KVFULL1, B_KVEMPTY0, B_KVEMPTY1, B_SFULL0,
+       B_SFULL1, B_SEMPTY0, B_SEMPTY1, B_PFULL, B_PEMPTY, B_OFULL, B_DRAIN, B_COUNT };
 
 struct Item {
   int tok0, L, K, kvh, branch, row0, q0, nrows, n_prefix_tiles, n_tiles;
@@ -100,7 +105,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
     for (int i = 0; i < B_COUNT; ++i) {
-      const uint32_t cnt = (i == B_SEMPTY0 || i == B_SEMPTY1 || i == B_PFULL) ? 128u : 1u;
+      const uint32_t cnt = (i == B_SEMPTY0 || i == B_SEMPTY1 || i == B_PFULL) ? (uint32_t)kSoftmax : 1u;
       mbar_init(bar(i), cnt);
     }
     fence_barrier_init();
@@ -115,20 +120,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_holder;
   const uint32_t tmemO = tmem + 256;
 
-  // running counts, identical in every role (same items, same tiles)
-  uint32_t n_item = 0, n_kv = 0, n_s = 0, n_p = 0;
-  bool ok = true;
-
-  for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++n_item) {
-    const Item m = load_item<G>(plan, it, b);
-    if (warp == 0) {
-      if (lane == 0 && ok) {
-        mbar_arrive_expect_tx(bar(B_QFULL), 2 * kHalf);
+  // Every role walks the same items and tiles, so the running counts below
+  // (items, KV tiles, S buffers, P buffers) agree across roles and give each
+  // barrier's phase.  Roles run ahead of each other across item boundaries.
+  if (warp == 0) {
+    // ---- TMA producer
+    if (lane == 0) {
+      uint32_t n_kv = 0, n_item = 0;
+      for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++n_item) {
+        const Item m = load_item<G>(plan, it, b);
+        const uint32_t qs = n_item & 1, quse = n_item >> 1;
+        if (!mbar_wait(bar(B_QEMPTY0 + qs), (quse & 1u) ^ 1u, st, 40)) break;
+        mbar_arrive_expect_tx(bar(B_QFULL0 + qs), 2 * kHalf);
         for (int h = 0; h < 2; ++h)
-          tma_load_3d(&tmQ, sbase + kQOff + h * kHalf, bar(B_QFULL), h * 64, m.kvh * G, m.tok0 + m.q0);
-        for (int t = 0; t < m.n_tiles && ok; ++t) {
-          const uint32_t slot = (n_kv + t) & 1, use = (n_kv + t) >> 1;
-          if (!mbar_wait(bar(B_KVEMPTY0 + slot), (use & 1u) ^ 1u, st, 40)) {
+          tma_load_3d(&tmQ, sbase + kQOff + (2 * qs + h) * kHalf, bar(B_QFULL0 + qs), h * 64, m.kvh * G,
+                      m.tok0 + m.q0);
+        bool ok = true;
+        for (int t = 0; t < m.n_tiles; ++t, ++n_kv) {
+          const uint32_t slot = n_kv & 1, use = n_kv >> 1;
+          if (!mbar_wait(bar(B_KVEMPTY0 + slot), (use & 1u) ^ 1u, st, 41)) {
             ok = false;
             break;
           }
@@ -139,11 +149,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(&tmV, sbase + kVOff + (2 * slot + h) * kHalf, bar(B_KVFULL0 + slot), h * 64, y);
           }
         }
+        if (!ok) break;
       }
-    } else if (warp == 1) {
-      if (lane == 0 && ok) {
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer
+    if (lane == 0) {
+      uint32_t n_kv = 0, n_s = 0, n_p = 0, n_item = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++n_item) {
+        const Item m = load_item<G>(plan, it, b);
+        const uint32_t qs = n_item & 1, quse = n_item >> 1;
         auto pv = [&](int t) -> bool {
-          if (!mbar_wait(bar(B_PFULL), (n_p + t) & 1u, st, 41)) return false;
+          if (!mbar_wait(bar(B_PFULL), (n_p + t) & 1u, st, 42)) return false;
           tc_fence_after();
           const uint32_t slot = (n_kv + t) & 1;
 #pragma unroll
@@ -156,55 +174,88 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_commit(bar(B_PEMPTY));
           return true;
         };
-        if (!mbar_wait(bar(B_QFULL), n_item & 1u, st, 42)) ok = false;
+        if (!mbar_wait(bar(B_QFULL0 + qs), quse & 1u, st, 43)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         for (int t = 0; t < m.n_tiles && ok; ++t) {
           const uint32_t slot = (n_kv + t) & 1, kuse = (n_kv + t) >> 1;
           const uint32_t sb = (n_s + t) & 1, suse = (n_s + t) >> 1;
-          if (!mbar_wait(bar(B_KVFULL0 + slot), kuse & 1u, st, 43) ||
-              !mbar_wait(bar(B_SEMPTY0 + sb), (suse & 1u) ^ 1u, st, 44)) {
+          if (!mbar_wait(bar(B_KVFULL0 + slot), kuse & 1u, st, 44) ||
+              !mbar_wait(bar(B_SEMPTY0 + sb), (suse & 1u) ^ 1u, st, 45)) {
             ok = false;
             break;
           }
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < kHD / 16; ++k) {
-            const uint64_t da = smem_desc_sw128(sbase + kQOff + (k >> 2) * kHalf + (k & 3) * 32);
+            const uint64_t da = smem_desc_sw128(sbase + kQOff + (2 * qs + (k >> 2)) * kHalf + (k & 3) * 32);
             const uint64_t db = smem_desc_sw128(sbase + kKOff + (2 * slot + (k >> 2)) * kHalf + (k & 3) * 32);
             tc_mma_f16(tmem + sb * kKeys, da, db, kIdescS, k > 0 ? 1u : 0u);
           }
           tc_commit(bar(B_SFULL0 + sb));
+          if (t == m.n_tiles - 1) tc_commit(bar(B_QEMPTY0 + qs));  // Q slot free once these S are done
           if (t > 0 && !pv(t - 1)) ok = false;
         }
         if (ok && !pv(m.n_tiles - 1)) ok = false;
         if (ok) tc_commit(bar(B_OFULL));
+        n_kv += m.n_tiles;
+        n_s += m.n_tiles;
+        n_p += m.n_tiles;
       }
-    } else {
-      // ---- softmax: thread = slot row r = TMEM lane
-      const int q4 = warp & 3;
-      const int r = q4 * 32 + lane;
-      const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+      // no tensor-core operation of this CTA may outlive its TMEM
+      tc_commit(bar(B_DRAIN));
+      mbar_wait(bar(B_DRAIN), 0, st, 46);
+    }
+  } else {
+    // ---- softmax: thread = (slot row r = TMEM lane, column half ch); the two
+    // threads of a row exchange partial maxima (and at the end the sums)
+    // through shared memory
+    const int q4 = warp & 3;
+    const int ch = (warp - 2) >> 2;  // 0: keys / dims [0, 64), 1: [64, 128)
+    const int r = q4 * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    float* red = reinterpret_cast<float*>(smem + kRedOff);  // [2][128]
+    // Barrier over the softmax threads that also ANDs a flag across them, so
+    // that a failed (timed-out) wait stops all eight warps together and none
+    // is left at a named barrier.
+    auto softmax_all = [](bool v) -> bool {
+      uint32_t res;
+      asm volatile(
+          "{ .reg .pred pin, pout; setp.ne.u32 pin, %1, 0; bar.red.and.pred pout, 1, %2, pin; "
+          "selp.u32 %0, 1, 0, pout; }"
+          : "=r"(res)
+          : "r"(v ? 1u : 0u), "n"(kSoftmax)
+          : "memory");
+      return res != 0;
+    };
+    uint32_t n_s = 0, n_p = 0, n_item = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++n_item) {
+      const Item m = load_item<G>(plan, it, b);
       const KeyRange kr = tree_keys(m.q0 + r / G, m.L, b);
       float m_used = -INFINITY, l = 0.f;
       for (int t = 0; t < m.n_tiles && ok; ++t) {
         const uint32_t sb = (n_s + t) & 1, suse = (n_s + t) >> 1;
-        if (!mbar_wait_warp(bar(B_SFULL0 + sb), suse & 1u, st, 45)) {
+        if (!softmax_all(mbar_wait_warp(bar(B_SFULL0 + sb), suse & 1u, st, 47))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const int k0 = m.tile_start(t);
+        const int k0 = m.tile_start(t) + 64 * ch;
         const bool is_branch_tile = m.branch && t == m.n_prefix_tiles;
-        const bool need_mask = is_branch_tile || (!m.branch && k0 + kKeys > m.row0) || (m.branch && k0 + kKeys > m.L);
-        const uint32_t s_addr = tmem + lane_off + sb * kKeys;
-        // the whole S row in registers: four loads, one wait
-        uint32_t sr[4][32];
+        const bool need_mask = is_branch_tile || (!m.branch && m.tile_start(t) + kKeys > m.row0) ||
+                               (m.branch && m.tile_start(t) + kKeys > m.L);
+        const uint32_t s_addr = tmem + lane_off + sb * kKeys + 64 * ch;
+        // this thread's 64 S values: two loads, one wait
+        uint32_t sr[2][32];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_ld32_async(s_addr + 32 * q, sr[q]);
+        for (int q = 0; q < 2; ++q) tmem_ld32_async(s_addr + 32 * q, sr[q]);
         tmem_wait_ld();
         float mx = -INFINITY;
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
+        for (int q = 0; q < 2; ++q)
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             tmem_ld_fence(sr[q][j]);
@@ -217,22 +268,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             sr[q][j] = __float_as_uint(x);
             mx = fmaxf(mx, x);
           }
-        // P buffer free and O complete for the previous tile
-        if (!mbar_wait_warp(bar(B_PEMPTY), ((n_p + t) & 1u) ^ 1u, st, 46)) {
+        // S buffer consumed: the MMA may refill it
+        tc_fence_before();
+        mbar_arrive(bar(B_SEMPTY0 + sb));
+        // row max over both halves; the barrier that publishes the partial
+        // maxima also confirms the P buffer is free and O complete for the
+        // previous tile (the next tile's writes of red[] come after its first
+        // barrier, which every thread reaches only after reading red[] here)
+        red[ch * 128 + r] = mx;
+        if (!softmax_all(mbar_wait_warp(bar(B_PEMPTY), ((n_p + t) & 1u) ^ 1u, st, 48))) {
           ok = false;
           break;
         }
+        mx = fmaxf(mx, red[(ch ^ 1) * 128 + r]);
         tc_fence_after();
         const float m_new = fmaxf(m_used, mx);
         // the O rescale uses warp-collective TMEM loads and stores: decide it
-        // for the whole warp (a row that did not need it is rescaled to its
+        // for the whole warp (both warps of a row group see the same maxima,
+        // so they decide alike; a row that did not need it is rescaled to its
         // new max as well, which is just as exact)
         if (t == 0) {
           m_used = m_new;
         } else if (__any_sync(0xffffffffu, m_new > m_used + kRescaleLog2)) {
           const float corr = m_new == m_used ? 1.f : fast_exp2(m_used - m_new);  // 0 while nothing was visible
 #pragma unroll 1
-          for (int c = 0; c < kHD; c += 32) {
+          for (int c = 64 * ch; c < 64 * ch + 64; c += 32) {
             float v[32];
             tmem_ld32(tmemO + lane_off + c, v);
 #pragma unroll
@@ -243,23 +303,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_used = m_new;
         }
         const float mu = m_used == -INFINITY ? 0.f : m_used;
-        // P = 2^(s - mu) in fp16, K-major 128-byte-swizzled rows
+        // P = 2^(s - mu) in fp16 into this half's K-major 128-byte-swizzled box
         float sum = 0.f;
+        const uint32_t pbox = sbase + kPOff + ch * kHalf + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 2; ++q) {
           uint32_t pk[16];
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
-            const __half2 h = __floats2half2_rn(fast_exp2(__uint_as_float(sr[q][j]) - mu),
-                                                fast_exp2(__uint_as_float(sr[q][j + 1]) - mu));
-            const float2 hf = __half22float2(h);  // sum what the tensor core will see
-            sum += hf.x + hf.y;
+            const float p0 = fast_exp2(__uint_as_float(sr[q][j]) - mu);
+            const float p1 = fast_exp2(__uint_as_float(sr[q][j + 1]) - mu);
+            sum += p0 + p1;
+            const __half2 h = __floats2half2_rn(p0, p1);
             pk[j / 2] = *reinterpret_cast<const uint32_t*>(&h);
           }
-          const uint32_t pbox = sbase + kPOff + (q >> 1) * kHalf + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int chunk = (q & 1) * 4 + u;
+            const int chunk = q * 4 + u;
             asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(pbox + ((chunk ^ (r & 7)) << 4)),
                          "r"(pk[4 * u]), "r"(pk[4 * u + 1]), "r"(pk[4 * u + 2]), "r"(pk[4 * u + 3])
                          : "memory");
@@ -267,45 +327,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         l += sum;
         tc_fence_before();
-        mbar_arrive(bar(B_SEMPTY0 + sb));
         fence_proxy_async_smem();
         mbar_arrive(bar(B_PFULL));
       }
-      // ---- epilogue: O / l -> fp16
-      if (ok && mbar_wait_warp(bar(B_OFULL), n_item & 1u, st, 47)) {
-        tc_fence_after();
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        const int rl = r / G;
-        const bool valid = rl < m.nrows;
-        __half* dst = o + (((int64_t)m.tok0 + m.q0 + rl) * n_q_heads + m.kvh * G + (r % G)) * kHD;
-#pragma unroll 1
-        for (int c = 0; c < kHD; c += 32) {
-          float v[32];
-          tmem_ld32(tmemO + lane_off + c, v);
-          if (valid) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const __half2 h = __floats2half2_rn(v[2 * j] * inv, v[2 * j + 1] * inv);
-              pk[j] = *reinterpret_cast<const uint32_t*>(&h);
-            }
-            uint4* p = reinterpret_cast<uint4*>(dst + c);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) p[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-          }
-        }
-        tc_fence_before();
-      } else {
+      // ---- epilogue: O / l -> fp16, this thread's 64 dims (O is
+      // overwritten only after the next item's first P, which these warps
+      // release after this read)
+      if (!ok) break;
+      // (this barrier also orders the partner's read of the last partial
+      // max before the sum overwrites it)
+      if (!softmax_all(mbar_wait_warp(bar(B_OFULL), n_item & 1u, st, 49))) {
         ok = false;
+        break;
       }
+      tc_fence_after();
+      red[ch * 128 + r] = l;
+      asm volatile("bar.sync 1, %0;" ::"n"(kSoftmax) : "memory");
+      l += red[(ch ^ 1) * 128 + r];
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const int rl = r / G;
+      const bool valid = rl < m.nrows;
+      __half* dst = o + (((int64_t)m.tok0 + m.q0 + rl) * n_q_heads + m.kvh * G + (r % G)) * kHD;
+#pragma unroll 1
+      for (int c = 64 * ch; c < 64 * ch + 64; c += 32) {
+        float v[32];
+        tmem_ld32(tmemO + lane_off + c, v);
+        if (valid) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const __half2 h = __floats2half2_rn(v[2 * j] * inv, v[2 * j + 1] * inv);
+            pk[j] = *reinterpret_cast<const uint32_t*>(&h);
+          }
+          uint4* p = reinterpret_cast<uint4*>(dst + c);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) p[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+      }
+      tc_fence_before();
+      n_s += m.n_tiles;
+      n_p += m.n_tiles;
     }
-    n_kv += m.n_tiles;
-    n_s += m.n_tiles;
-    n_p += m.n_tiles;
-    // every async operation of this item is complete (the epilogue saw O):
-    // Q, the KV slots and O can be reused by the next item; a failed wait in
-    // any thread stops the whole CTA
-    if (__syncthreads_or(ok ? 0 : 1)) break;
   }
 
   tc_fence_before();
