@@ -126,6 +126,74 @@ __global__ void __launch_bounds__(kRowThreads)
   }
 }
 
+// fp16 path: the same gather, but the layer-0 norm is left to the QKV
+// epilogue: writes x, fp16(x * gain) and the row's sum of x^2 (slot 0; the
+// other n_slots - 1 partial-sum slots of the row are zeroed).
+template <int CH>
+__global__ void __launch_bounds__(kRowThreads)
+    embed_gain_kernel(const PlanHdr* __restrict__ plan, const void* __restrict__ embed,
+                      const __half* __restrict__ table, int64_t n_table, int vocab, int d,
+                      const float* __restrict__ gain, float* __restrict__ x, __half* __restrict__ xg,
+                      float* __restrict__ ssp, int n_slots, DevStatus* st) {
+  const int T = plan->n_tokens;
+  const int* ids = plan_array<int32_t>(plan, plan->off_ids);
+  const int lane = threadIdx.x & 31;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nw) {
+    const int id = ids[t];
+    float v[CH][8];
+    const bool ok = id >= 0 && (int64_t)id < (int64_t)vocab + n_table;
+    if (!ok && lane == 0) raise_error(st, ERR_BAD_INDEX, 33);
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const int col = (lane + 32 * c) * 8;
+      if (!ok || col >= d) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[c][i] = 0.f;
+      } else if (id >= vocab) {
+        load8_f16(table + (int64_t)(id - vocab) * d + col, v[c]);
+      } else {
+        load8_bf16(reinterpret_cast<const __nv_bfloat16*>(embed) + (int64_t)id * d + col, v[c]);
+      }
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const int col = (lane + 32 * c) * 8;
+      if (col >= d) continue;
+      float gv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        ss += v[c][i] * v[c][i];
+        gv[i] = v[c][i] * gain[col + i];
+      }
+      store8<float>(x + (int64_t)t * d + col, v[c], st);
+      store8<__half>(xg + (int64_t)t * d + col, gv, st);
+    }
+    ss = warp_sum(ss);
+    if (lane < n_slots) ssp[(int64_t)t * n_slots + lane] = lane == 0 ? ss : 0.f;
+  }
+}
+
+cudaError_t embed_gain(const PlanHdr* plan, const void* embed, const __half* table, int64_t n_table, int vocab, int d,
+                       const float* gain, float* x, __half* xg, float* ssp, int n_slots, DevStatus* st, int max_rows,
+                       cudaStream_t s) {
+  const int g = std::max(1, std::min((max_rows + 7) / 8, kMaxRowBlocks));
+  if (d % 8 || n_slots > 32 || n_slots % 4) return cudaErrorInvalidValue;
+  switch ((d + 255) / 256) {
+#define DUOLM_EG_CASE(n)                                                                                            \
+  case n:                                                                                                           \
+    embed_gain_kernel<n><<<g, kRowThreads, 0, s>>>(plan, embed, table, n_table, vocab, d, gain, x, xg, ssp, n_slots, \
+                                                   st);                                                             \
+    break;
+    DUOLM_EG_CASE(1) DUOLM_EG_CASE(2) DUOLM_EG_CASE(3) DUOLM_EG_CASE(4) DUOLM_EG_CASE(8)
+#undef DUOLM_EG_CASE
+    default:
+      return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
 template <typename OutT, int CH>
 __global__ void __launch_bounds__(kRowThreads)
     rmsnorm_kernel(const PlanHdr* __restrict__ plan, const float* __restrict__ x, int d,
@@ -206,12 +274,8 @@ cudaError_t rmsnorm_rows(const PlanHdr* plan, const float* x, int d, const float
   return cudaGetLastError();
 }
 
-template cudaError_t embed_norm<__half>(const PlanHdr*, const void*, bool, const __half*, int64_t, int, int,
-                                       const float*, float, float*, __half*, DevStatus*, int, cudaStream_t);
 template cudaError_t embed_norm<float>(const PlanHdr*, const void*, bool, const __half*, int64_t, int, int,
                                        const float*, float, float*, float*, DevStatus*, int, cudaStream_t);
-template cudaError_t rmsnorm_rows<__half>(const PlanHdr*, const float*, int, const float*, float, __half*,
-                                          DevStatus*, int, cudaStream_t);
 template cudaError_t rmsnorm_rows<float>(const PlanHdr*, const float*, int, const float*, float, float*,
                                          DevStatus*, int, cudaStream_t);
 

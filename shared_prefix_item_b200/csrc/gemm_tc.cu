@@ -44,13 +44,28 @@ __device__ __forceinline__ float silu_fast(float g) {
   return __fdividef(g, 1.0f + fast_exp2(-1.4426950408889634f * g));
 }
 
+// r = 1 / sqrt(mean(x^2) + eps) of one input row from its partial sums
+__device__ __forceinline__ float row_rnorm(const float* ssp, int n_slots, int row, float inv_d, float eps) {
+  const float4* p = reinterpret_cast<const float4*>(ssp + (int64_t)row * n_slots);
+  float ss = 0.f;
+  for (int i = 0; i < n_slots / 4; ++i) {
+    const float4 v = p[i];
+    ss += v.x;
+    ss += v.y;
+    ss += v.z;
+    ss += v.w;
+  }
+  return 1.0f / sqrtf(ss * inv_d + eps);
+}
+
 struct EpiResid {
   EpiResidArgs a;
   static constexpr int EG = 4;
   template <int BN>
   __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, int g, bool row_ok, const PlanHdr*,
-                                      DevStatus*) const {
+                                      DevStatus* st) const {
     constexpr int W = BN / EG;
+    float ss = 0.f;
 #pragma unroll 1
     for (int c = g * W; c < (g + 1) * W; c += 32) {
       float v[32];
@@ -68,8 +83,29 @@ struct EpiResid {
           t[j].w += v[4 * j + 3] * a.scale;
           p[j] = t[j];
         }
+        if (a.xg) {
+          const float* gn = a.g_next + n0 + c;
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            ss += t[j].x * t[j].x;
+            ss += t[j].y * t[j].y;
+            ss += t[j].z * t[j].z;
+            ss += t[j].w * t[j].w;
+            const __half2 h0 = __halves2half2(to_half_checked(t[j].x * gn[4 * j + 0], st, 23),
+                                              to_half_checked(t[j].y * gn[4 * j + 1], st, 23));
+            const __half2 h1 = __halves2half2(to_half_checked(t[j].z * gn[4 * j + 2], st, 23),
+                                              to_half_checked(t[j].w * gn[4 * j + 3], st, 23));
+            pk[2 * j] = *reinterpret_cast<const uint32_t*>(&h0);
+            pk[2 * j + 1] = *reinterpret_cast<const uint32_t*>(&h1);
+          }
+          uint4* q = reinterpret_cast<uint4*>(a.xg + (int64_t)row * a.ldx + n0 + c);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) q[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        }
       }
     }
+    if (row_ok && a.xg) a.ssp[(int64_t)row * a.n_slots + (n0 / BN) * EG + g] = ss;
   }
 };
 
@@ -82,6 +118,7 @@ struct EpiSwiglu {
     constexpr int H = BN / 2;   // gate columns [0, H), up columns [H, BN)
     constexpr int W = H / EG;   // outputs of this group
     const int out0 = n0 / 2;
+    const float sc = row_ok ? a.scale * row_rnorm(a.ssp, a.n_slots, row, a.inv_d, a.eps) : 0.f;
 #pragma unroll 1
     for (int c = g * W; c < (g + 1) * W; c += 32) {
       float gv[32], uv[32];
@@ -91,8 +128,8 @@ struct EpiSwiglu {
         uint32_t packed[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const float h0 = silu_fast(gv[2 * j] * a.scale) * (uv[2 * j] * a.scale);
-          const float h1 = silu_fast(gv[2 * j + 1] * a.scale) * (uv[2 * j + 1] * a.scale);
+          const float h0 = silu_fast(gv[2 * j] * sc) * (uv[2 * j] * sc);
+          const float h1 = silu_fast(gv[2 * j + 1] * sc) * (uv[2 * j + 1] * sc);
           __half2 hh = __halves2half2(to_half_checked(h0, st, 20), to_half_checked(h1, st, 20));
           packed[j] = *reinterpret_cast<uint32_t*>(&hh);
         }
@@ -115,6 +152,8 @@ struct EpiQkv {
                                       DevStatus* st) const {
     const int gc = n0 + 128 * g;
     const uint32_t base = taddr + 128 * g;
+    // weight scale times the input row's RMSNorm factor
+    const float sc = row_ok ? a.scale * row_rnorm(a.ssp, a.n_slots, row, a.inv_d, a.norm_eps) : 0.f;
     if (gc >= a.qd + a.kd) {  // value head
       const int head = (gc - a.qd - a.kd) >> 7;
       __half* dst = a.vc + ((int64_t)head * a.kv_rows + row) * 128;
@@ -126,8 +165,8 @@ struct EpiQkv {
           uint32_t pk[8];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            __half2 hh = __halves2half2(to_half_checked(v[2 * j] * a.scale, st, 21),
-                                        to_half_checked(v[2 * j + 1] * a.scale, st, 21));
+            __half2 hh = __halves2half2(to_half_checked(v[2 * j] * sc, st, 21),
+                                        to_half_checked(v[2 * j + 1] * sc, st, 21));
             pk[j] = *reinterpret_cast<uint32_t*>(&hh);
           }
           uint4* p = reinterpret_cast<uint4*>(dst + c);
@@ -149,7 +188,7 @@ struct EpiQkv {
       tmem_ld16(base + c, v);
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const float t = v[j] * a.scale;
+        const float t = v[j] * sc;
         ss += t * t;
       }
     }
@@ -176,8 +215,8 @@ struct EpiQkv {
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int i = c + j + e;
-            const float a1 = (x1[j + e] * a.scale * r) * gain[i];
-            const float a2 = (x2[j + e] * a.scale * r) * gain[64 + i];
+            const float a1 = (x1[j + e] * sc * r) * gain[i];
+            const float a2 = (x2[j + e] * sc * r) * gain[64 + i];
             const float2 t = cs[(int64_t)i * a.max_pos];
             r1[e] = a1 * t.x - a2 * t.y;
             r2[e] = a2 * t.x + a1 * t.y;

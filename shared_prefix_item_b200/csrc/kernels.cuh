@@ -8,15 +8,27 @@ namespace duolm {
 // ---- tcgen05 GEMM:  C[M, N] = A[M, K] * B[N, K]^T, fp16 operands, fp32 accumulate.
 // M is the batch's token count, read on the device from the plan.
 
+// The normed operand of the QKV and gate/up projections is carried as
+// xg = fp16(x * g) (g: the norm's gain) plus per-row partial sums of x^2 in
+// `ssp` ([rows][n_slots], one writer per slot); the consuming epilogue scales
+// its accumulator row by r = 1 / sqrt(sum(ssp) / d + eps), since
+// RMSNorm(x) * g * W = r * ((x * g) * W).
 struct EpiResidArgs {   // x[row][col] += scale * acc  (fp32 residual stream)
   float* x;
   int ldx;
   float scale;
+  __half* xg;           // optional: fp16(x * g_next) for the next projection
+  const float* g_next;  // gain of the next RMSNorm
+  float* ssp;           // partial sums of x^2: slot n_blk * 4 + group of the tile's columns
+  int n_slots;
 };
 struct EpiSwigluArgs {  // tile columns [0, BN/2) gate, [BN/2, BN) up -> h = silu(g) * u, fp16
   __half* h;
   int ldh;
   float scale;
+  const float* ssp;     // partial sums of x^2 of the input rows
+  int n_slots;
+  float inv_d, eps;
 };
 struct EpiQkvArgs {     // per 128-wide head: q/k RMSNorm + RoPE, v copy; fp16 out
   __half* q;            // [T][n_q_heads][128]
@@ -30,6 +42,9 @@ struct EpiQkvArgs {     // per 128-wide head: q/k RMSNorm + RoPE, v copy; fp16 o
   float scale;
   float eps;
   int qd, kd, n_q_heads;
+  const float* ssp;     // partial sums of x^2 of the input rows
+  int n_slots;
+  float inv_d, norm_eps;
 };
 
 bool make_tmap_f16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
@@ -54,6 +69,10 @@ template <typename OutT>
 cudaError_t embed_norm(const PlanHdr* plan, const void* embed, bool embed_bf16, const __half* table,
                        int64_t n_table, int vocab, int d, const float* gain, float eps, float* x, OutT* xn,
                        DevStatus* st, int max_rows, cudaStream_t s);
+// fp16 path: gather into x, write fp16(x * gain) and the row's sum of x^2
+cudaError_t embed_gain(const PlanHdr* plan, const void* embed, const __half* table, int64_t n_table, int vocab, int d,
+                       const float* gain, float* x, __half* xg, float* ssp, int n_slots, DevStatus* st, int max_rows,
+                       cudaStream_t s);
 template <typename OutT>
 cudaError_t rmsnorm_rows(const PlanHdr* plan, const float* x, int d, const float* gain, float eps, OutT* xn,
                          DevStatus* st, int max_rows, cudaStream_t s);
@@ -70,14 +89,9 @@ cudaError_t debug_wait_timeout(DevStatus* st, cudaStream_t s);
 cudaError_t debug_mask(const PlanHdr* plan, int request, uint8_t* out, int64_t tq, cudaStream_t s);
 
 // ---- attention
-cudaError_t attention_f16(const PlanHdr* plan, const __half* q, const __half* kc, const __half* vc,
-                          int64_t kv_rows, int n_q_heads, int n_kv_heads, float scale, __half* o, DevStatus* st,
-                          int grid, cudaStream_t s);
 cudaError_t attention_f32(const PlanHdr* plan, const float* q, const float* kc, const float* vc, int64_t kv_rows,
                           int n_q_heads, int n_kv_heads, int hd, float scale, float* o, int max_rows,
                           cudaStream_t s);
-int attention_rows_per_item(int group);
-cudaError_t attention_setup();
 // tcgen05 attention (fp16 path): items of 128 query slots, KV tiles of 128 keys
 cudaError_t attention_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const PlanHdr* plan,
                          int64_t kv_rows, int n_q_heads, int n_kv_heads, float scale, __half* o, DevStatus* st,

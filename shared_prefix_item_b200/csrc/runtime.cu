@@ -77,6 +77,7 @@ struct duolm_ctx {
   void* h = nullptr;
   float* qkv32 = nullptr;
   float* gu32 = nullptr;
+  float* ssp = nullptr;  // fp16 path: per-row partial sums of x^2 [T][d / 64]
   float* scores = nullptr;
   char* plan_dev = nullptr;
   char* plan_host = nullptr;
@@ -224,6 +225,7 @@ void free_workspace(duolm_ctx* c) {
   dfree(c->h);
   dfree(c->qkv32);
   dfree(c->gu32);
+  dfree(c->ssp);
   dfree(c->scores);
   dfree(c->plan_dev);
   if (c->plan_host) cudaFreeHost(c->plan_host);
@@ -272,7 +274,9 @@ int reserve_impl(duolm_ctx* ctx, int64_t T, int64_t R, int64_t C) {
   CK(cudaMemset(ctx->vc, 0, d.n_kv_heads * kv_rows * d.head_dim * es));
   if ((rc = dalloc(ctx, &ctx->o, T * ctx->qd * es))) return rc;
   if ((rc = dalloc(ctx, &ctx->h, T * d.ffn * es))) return rc;
-  if (!ctx->f16) {
+  if (ctx->f16) {
+    if ((rc = dalloc(ctx, &ctx->ssp, T * (d.d / 64) * 4))) return rc;
+  } else {
     if ((rc = dalloc(ctx, &ctx->qkv32, T * (ctx->qd + 2 * ctx->kd) * 4))) return rc;
     if ((rc = dalloc(ctx, &ctx->gu32, T * 2 * d.ffn * 4))) return rc;
   }
@@ -340,27 +344,35 @@ cudaError_t launch_forward(duolm_ctx* c, int n_layers, bool with_head, int64_t* 
   const float attn_scale = 1.0f / sqrtf((float)d.head_dim);
   int64_t launches = 0;
   if (c->f16) {
-    __half* xn = static_cast<__half*>(c->xn);
-    LCK(DUOLM_PROF_EMBED, embed_norm<__half>(plan, c->embed, true, c->table, c->n_items, d.vocab, d.d, c->gains + c->layers[0].g_attn,
-                           d.rms_eps, c->x, xn, c->status, maxT, s));
+    // RMSNorm is folded into the projections: x's producer writes
+    // fp16(x * g) and per-row partial sums of x^2, the consuming epilogue
+    // scales its rows by 1 / sqrt(mean(x^2) + eps)
+    __half* xg = static_cast<__half*>(c->xn);
+    const int n_slots = d.d / 64;
+    const float inv_d = 1.0f / (float)d.d;
+    LCK(DUOLM_PROF_EMBED, embed_gain(plan, c->embed, c->table, c->n_items, d.vocab, d.d, c->gains + c->layers[0].g_attn,
+                                     c->x, xg, c->ssp, n_slots, c->status, maxT, s));
     for (int l = 0; l < n_layers; ++l) {
       const LayerW& L = c->layers[l];
       EpiQkvArgs qa{static_cast<__half*>(c->q), static_cast<__half*>(c->kc), static_cast<__half*>(c->vc), c->rope,
                     kv_rows, kMaxPos, c->gains + L.g_q, c->gains + L.g_k, L.s_qkv, d.rms_eps, c->qd, c->kd,
-                    d.n_q_heads};
+                    d.n_q_heads, c->ssp, n_slots, inv_d, d.rms_eps};
       LCK(DUOLM_PROF_GEMM_QKV, gemm_tc_qkv(c->tm_xn, L.tm_qkv, d.d, c->qd + 2 * c->kd, plan, qa, c->status, c->num_sms, s));
       LCK(DUOLM_PROF_ATTENTION, attention_tc(c->tm_q3, c->tm_kc, c->tm_vc, plan, kv_rows, d.n_q_heads, d.n_kv_heads,
                                              attn_scale, static_cast<__half*>(c->o), c->status, c->num_sms, s));
-      LCK(DUOLM_PROF_GEMM_O, gemm_tc_resid(c->tm_oact, L.tm_o, c->qd, d.d, plan, EpiResidArgs{c->x, d.d, L.s_o}, c->status,
-                        c->num_sms, s));
-      LCK(DUOLM_PROF_RMSNORM, rmsnorm_rows<__half>(plan, c->x, d.d, c->gains + L.g_mlp, d.rms_eps, xn, c->status, maxT, s));
-      LCK(DUOLM_PROF_GEMM_GATE_UP, gemm_tc_swiglu(c->tm_xn, L.tm_gu, d.d, 2 * d.ffn, plan,
-                         EpiSwigluArgs{static_cast<__half*>(c->h), d.ffn, L.s_gu}, c->status, c->num_sms, s));
-      LCK(DUOLM_PROF_GEMM_DOWN, gemm_tc_resid(c->tm_h, L.tm_d, d.ffn, d.d, plan, EpiResidArgs{c->x, d.d, L.s_d}, c->status, c->num_sms,
-                        s));
-      if (l + 1 < n_layers)
-        LCK(DUOLM_PROF_RMSNORM, rmsnorm_rows<__half>(plan, c->x, d.d, c->gains + c->layers[l + 1].g_attn, d.rms_eps, xn, c->status,
-                                 maxT, s));
+      LCK(DUOLM_PROF_GEMM_O, gemm_tc_resid(c->tm_oact, L.tm_o, c->qd, d.d, plan,
+                                           EpiResidArgs{c->x, d.d, L.s_o, xg, c->gains + L.g_mlp, c->ssp, n_slots},
+                                           c->status, c->num_sms, s));
+      LCK(DUOLM_PROF_GEMM_GATE_UP,
+          gemm_tc_swiglu(c->tm_xn, L.tm_gu, d.d, 2 * d.ffn, plan,
+                         EpiSwigluArgs{static_cast<__half*>(c->h), d.ffn, L.s_gu, c->ssp, n_slots, inv_d, d.rms_eps},
+                         c->status, c->num_sms, s));
+      const bool last = l + 1 == n_layers;
+      LCK(DUOLM_PROF_GEMM_DOWN,
+          gemm_tc_resid(c->tm_h, L.tm_d, d.ffn, d.d, plan,
+                        EpiResidArgs{c->x, d.d, L.s_d, last ? nullptr : xg,
+                                     last ? nullptr : c->gains + c->layers[l + 1].g_attn, c->ssp, n_slots},
+                        c->status, c->num_sms, s));
     }
   } else {
     float* xn = static_cast<float*>(c->xn);
@@ -944,7 +956,8 @@ int duolm_debug_gemm(duolm_ctx* ctx, int layer, int which, const uint16_t* a, fl
   cudaError_t e = cudaMemsetAsync(tmp, 0, T * N * 4, ctx->stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(abuf, a, T * K * 2, cudaMemcpyHostToDevice, ctx->stream);
   if (e == cudaSuccess)
-    e = gemm_tc_resid(ta, tb, K, N, reinterpret_cast<const PlanHdr*>(ctx->plan_dev), EpiResidArgs{tmp, N, sc},
+    e = gemm_tc_resid(ta, tb, K, N, reinterpret_cast<const PlanHdr*>(ctx->plan_dev),
+                      EpiResidArgs{tmp, N, sc, nullptr, nullptr, nullptr, 0},
                       ctx->status, ctx->num_sms, ctx->stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(out, tmp, T * N * 4, cudaMemcpyDeviceToHost, ctx->stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(ctx->stream);
