@@ -22,16 +22,21 @@ namespace duolm {
 constexpr int kBM = 128;
 constexpr int kBK = 64;  // one 128-byte swizzle row of fp16
 
+// A CTA pair (cluster of 2) computes a 256 x BN tile: each CTA loads its 128
+// rows of A and its BN/2 rows of B per k-block (32 KB), the leader issues
+// the pair MMAs (M = 256), each CTA's TMEM receives its 128 accumulator rows.
+// Tiles are visited N-fastest, so the pairs running at the same time share
+// an A row block and it is read from DRAM once.
 template <int BN>
 struct TcCfg {
-  static constexpr int STAGES = BN == 256 ? 4 : 6;
-  static constexpr int A_BYTES = kBM * kBK * 2;
-  static constexpr int B_BYTES = BN * kBK * 2;
+  static constexpr int STAGES = 6;
+  static constexpr int A_BYTES = kBM * kBK * 2;        // this CTA's 128 rows of A
+  static constexpr int B_BYTES = (BN / 2) * kBK * 2;   // this CTA's half of the B tile
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-  static constexpr int SMEM = BAR_OFF + 256 + 1024;  // barriers + alignment slack
-  static constexpr uint32_t TMEM_COLS = 2 * BN;
-  static constexpr uint32_t IDESC = idesc_f16_f32(kBM, BN);
+  static constexpr int SMEM = BAR_OFF + 256 + 1024;    // barriers + alignment slack
+  static constexpr uint32_t TMEM_COLS = 2 * BN;        // two accumulator buffers
+  static constexpr uint32_t IDESC = idesc_f16_f32(2 * kBM, BN);
 };
 
 // ---------------------------------------------------------------------------
@@ -68,13 +73,23 @@ struct EpiResid {
     float ss = 0.f;
 #pragma unroll 1
     for (int c = g * W; c < (g + 1) * W; c += 32) {
-      float v[32];
-      tmem_ld32(taddr + c, v);
+      // the residual loads do not depend on the accumulator: issue them first
+      float4* p = reinterpret_cast<float4*>(a.x + (int64_t)(row_ok ? row : 0) * a.ldx + n0 + c);
+      float4 t[8];
       if (row_ok) {
-        float4* p = reinterpret_cast<float4*>(a.x + (int64_t)row * a.ldx + n0 + c);
-        float4 t[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) t[j] = p[j];
+      }
+      uint32_t vr[32];
+      tmem_ld32_async(taddr + c, vr);
+      tmem_wait_ld();
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        tmem_ld_fence(vr[j]);
+        v[j] = __uint_as_float(vr[j]);
+      }
+      if (row_ok) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           t[j].x += v[4 * j + 0] * a.scale;
@@ -121,9 +136,18 @@ struct EpiSwiglu {
     const float sc = row_ok ? a.scale * row_rnorm(a.ssp, a.n_slots, row, a.inv_d, a.eps) : 0.f;
 #pragma unroll 1
     for (int c = g * W; c < (g + 1) * W; c += 32) {
+      uint32_t gr[32], ur[32];
+      tmem_ld32_async(taddr + c, gr);
+      tmem_ld32_async(taddr + H + c, ur);
+      tmem_wait_ld();
       float gv[32], uv[32];
-      tmem_ld32(taddr + c, gv);
-      tmem_ld32(taddr + H + c, uv);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        tmem_ld_fence(gr[j]);
+        tmem_ld_fence(ur[j]);
+        gv[j] = __uint_as_float(gr[j]);
+        uv[j] = __uint_as_float(ur[j]);
+      }
       if (row_ok) {
         uint32_t packed[16];
 #pragma unroll
@@ -238,12 +262,13 @@ struct EpiQkv {
 };
 
 // ---------------------------------------------------------------------------
-// the kernel: warp 0 TMA producer, warp 1 MMA issuer, warps 2 .. 2 + 4*EG - 1
-// epilogue (group g = (warp - 2) / 4; each group spans the four TMEM lane
-// quadrants, warp w accessing lanes 32 * (w % 4) .. + 31)
+// the kernel, per CTA of a pair: warp 0 TMA producer, warp 1 TMEM allocation
+// and (leader only) the MMA issuer, warps 2 .. 2 + 4*EG - 1 epilogue (group
+// g = (warp - 2) / 4; each group spans the four TMEM lane quadrants, warp w
+// accessing lanes 32 * (w % 4) .. + 31)
 // ---------------------------------------------------------------------------
 template <int BN, class Epi>
-__global__ void __launch_bounds__(64 + 128 * Epi::EG, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 128 * Epi::EG, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int Kdim,
                    int N, const PlanHdr* __restrict__ plan, const Epi epi, DevStatus* st) {
   using C = TcCfg<BN>;
@@ -255,16 +280,19 @@ __global__ void __launch_bounds__(64 + 128 * Epi::EG, 1)
   const uint32_t empty0 = smem_u32(bars + C::STAGES);
   const uint32_t tfull0 = smem_u32(bars + 2 * C::STAGES);
   const uint32_t tempty0 = smem_u32(bars + 2 * C::STAGES + 2);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 4);
+  const uint32_t drain = smem_u32(bars + 2 * C::STAGES + 4);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 5);
+  uint32_t* skip_flag = tmem_holder + 1;
 
-  // a bounded wait already gave up in an earlier launch: do nothing
-  if (*reinterpret_cast<volatile const uint32_t*>(&st->flags) & ERR_WAIT_TIMEOUT) return;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int M = plan->n_tokens;
-  const int m_tiles = (M + kBM - 1) / kBM;
+  const int m_tiles = (M + 2 * kBM - 1) / (2 * kBM);
   const int n_tiles = N / BN;
   const int num_tiles = m_tiles * n_tiles;
   const int kblocks = Kdim / kBK;
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
 
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmA);
@@ -275,99 +303,116 @@ __global__ void __launch_bounds__(64 + 128 * Epi::EG, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull0 + 8 * a, 1);
-      mbar_init(tempty0 + 8 * a, 128 * EG);
+      mbar_init(tempty0 + 8 * a, 2 * 128 * EG);  // the epilogue threads of both CTAs
     }
+    mbar_init(drain, 1);
     fence_barrier_init();
+    // a bounded wait already gave up in an earlier launch: the pair skips its
+    // work, on the leader's reading of the flag so both CTAs agree
+    if (leader) *skip_flag = (*reinterpret_cast<volatile const uint32_t*>(&st->flags) & ERR_WAIT_TIMEOUT) ? 1u : 0u;
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  const bool skip = ld_shared_cluster_u32(map_to_rank(smem_u32(skip_flag), 0)) != 0;
 
-  if (warp == 0) {
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int m_blk = tile % m_tiles, n_blk = tile / m_tiles;
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, st, 1)) {
-            ok = false;
-            break;
-          }
-          const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
-          const uint32_t sb = sa + C::A_BYTES;
-          mbar_arrive_expect_tx(full0 + 8 * stage, C::STAGE_BYTES);
-          tma_load_2d(&tmA, sa, full0 + 8 * stage, kb * kBK, m_blk * kBM);
-          tma_load_2d(&tmB, sb, full0 + 8 * stage, kb * kBK, n_blk * BN);
-          if (++stage == C::STAGES) {
-            stage = 0;
-            phase ^= 1u;
+  if (!skip) {
+    if (warp == 0) {
+      if (lane == 0) {
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = pair; tile < num_tiles && ok; tile += n_pairs) {
+          const int m_blk = tile / n_tiles, n_blk = tile % n_tiles;
+          for (int kb = 0; kb < kblocks; ++kb) {
+            if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, st, 1)) {
+              ok = false;
+              break;
+            }
+            const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
+            const uint32_t sb = sa + C::A_BYTES;
+            // both CTAs' bytes complete on the leader's full barrier
+            const uint32_t full_leader = map_to_rank(full0 + 8 * stage, 0);
+            if (leader) mbar_arrive_expect_tx(full0 + 8 * stage, 2 * C::STAGE_BYTES);
+            tma_load_2d_pair(&tmA, sa, full_leader, kb * kBK, m_blk * 2 * kBM + (int)rank * kBM);
+            tma_load_2d_pair(&tmB, sb, full_leader, kb * kBK, n_blk * BN + (int)rank * (BN / 2));
+            if (++stage == C::STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
         }
       }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
+    } else if (warp == 1) {
+      if (lane == 0 && leader) {
+        int stage = 0;
+        uint32_t phase = 0;
+        int local = 0;
+        bool ok = true;
+        for (int tile = pair; tile < num_tiles && ok; tile += n_pairs, ++local) {
+          const int acc = local & 1;
+          const uint32_t use = (uint32_t)(local >> 1);
+          if (!mbar_wait(tempty0 + 8 * acc, (use & 1u) ^ 1u, st, 2)) break;
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + acc * BN;
+          for (int kb = 0; kb < kblocks; ++kb) {
+            if (!mbar_wait(full0 + 8 * stage, phase, st, 3)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
+            const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k) {
+              tc_mma_f16_pair(d_tmem, smem_desc_sw128(sa + 32 * k), smem_desc_sw128(sb + 32 * k), C::IDESC,
+                              (kb | k) != 0 ? 1u : 0u);
+            }
+            tc_commit_pair_both(empty0 + 8 * stage);
+            if (++stage == C::STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          if (ok) tc_commit_pair_both(tfull0 + 8 * acc);
+        }
+        // one more commit, observed by both CTAs before they leave: every
+        // earlier arrival of this pair's MMAs has landed by then
+        tc_commit_pair_both(drain);
+      }
+    } else {
+      const int q4 = warp & 3;            // TMEM lane quadrant this warp may access
+      const int group = (warp - 2) >> 2;  // column group of the tile
       int local = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+      for (int tile = pair; tile < num_tiles; tile += n_pairs, ++local) {
         const int acc = local & 1;
         const uint32_t use = (uint32_t)(local >> 1);
-        if (!mbar_wait(tempty0 + 8 * acc, (use & 1u) ^ 1u, st, 2)) break;
+        if (!mbar_wait_warp(tfull0 + 8 * acc, use & 1u, st, 4)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(full0 + 8 * stage, phase, st, 3)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
-          const uint32_t sb = sa + C::A_BYTES;
-#pragma unroll
-          for (int k = 0; k < kBK / 16; ++k) {
-            tc_mma_f16(d_tmem, smem_desc_sw128(sa + 32 * k), smem_desc_sw128(sb + 32 * k), C::IDESC,
-                       (kb | k) != 0 ? 1u : 0u);
-          }
-          tc_commit(empty0 + 8 * stage);
-          if (++stage == C::STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-        if (ok) tc_commit(tfull0 + 8 * acc);
+        const int m_blk = tile / n_tiles, n_blk = tile % n_tiles;
+        const int row = m_blk * 2 * kBM + (int)rank * kBM + q4 * 32 + lane;
+        const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q4 * 32) << 16);
+        epi.template run<BN>(taddr, row, n_blk * BN, group, row < M, plan, st);
+        // the accumulator may be overwritten once every epilogue thread of
+        // the pair has read it; the reads are ordered by the tcgen05 fence,
+        // the global stores need no ordering with the MMA
+        tc_fence_before();
+        mbar_arrive_cluster_relaxed(map_to_rank(tempty0 + 8 * acc, 0));
       }
     }
-  } else {
-    const int q4 = warp & 3;           // TMEM lane quadrant this warp may access
-    const int group = (warp - 2) >> 2;  // column group of the tile
-    int local = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
-      const int acc = local & 1;
-      const uint32_t use = (uint32_t)(local >> 1);
-      if (!mbar_wait_warp(tfull0 + 8 * acc, use & 1u, st, 4)) break;
-      tc_fence_after();
-      const int m_blk = tile % m_tiles, n_blk = tile / m_tiles;
-      const int row = m_blk * kBM + q4 * 32 + lane;
-      const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q4 * 32) << 16);
-      epi.template run<BN>(taddr, row, n_blk * BN, group, row < M, plan, st);
-      tc_fence_before();
-      mbar_arrive(tempty0 + 8 * acc);
-    }
+    if (threadIdx.x == 0) mbar_wait(drain, 0, st, 5);
   }
 
+  // no CTA leaves while its peer may still signal it or read its memory
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+  if (warp == 1) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
 }
 
 // ---------------------------------------------------------------------------

@@ -54,6 +54,7 @@ struct duolm_ctx {
   bool own_stream = false;
   bool f16 = false;
   int num_sms = 148;
+  int gemm_grid = 148;  // whole CTA pairs
   int qd = 0, kd = 0, group = 1, rows_per_item = 64;
 
   void* embed = nullptr;
@@ -357,22 +358,22 @@ cudaError_t launch_forward(duolm_ctx* c, int n_layers, bool with_head, int64_t* 
       EpiQkvArgs qa{static_cast<__half*>(c->q), static_cast<__half*>(c->kc), static_cast<__half*>(c->vc), c->rope,
                     kv_rows, kMaxPos, c->gains + L.g_q, c->gains + L.g_k, L.s_qkv, d.rms_eps, c->qd, c->kd,
                     d.n_q_heads, c->ssp, n_slots, inv_d, d.rms_eps};
-      LCK(DUOLM_PROF_GEMM_QKV, gemm_tc_qkv(c->tm_xn, L.tm_qkv, d.d, c->qd + 2 * c->kd, plan, qa, c->status, c->num_sms, s));
+      LCK(DUOLM_PROF_GEMM_QKV, gemm_tc_qkv(c->tm_xn, L.tm_qkv, d.d, c->qd + 2 * c->kd, plan, qa, c->status, c->gemm_grid, s));
       LCK(DUOLM_PROF_ATTENTION, attention_tc(c->tm_q3, c->tm_kc, c->tm_vc, plan, kv_rows, d.n_q_heads, d.n_kv_heads,
                                              attn_scale, static_cast<__half*>(c->o), c->status, c->num_sms, s));
       LCK(DUOLM_PROF_GEMM_O, gemm_tc_resid(c->tm_oact, L.tm_o, c->qd, d.d, plan,
                                            EpiResidArgs{c->x, d.d, L.s_o, xg, c->gains + L.g_mlp, c->ssp, n_slots},
-                                           c->status, c->num_sms, s));
+                                           c->status, c->gemm_grid, s));
       LCK(DUOLM_PROF_GEMM_GATE_UP,
           gemm_tc_swiglu(c->tm_xn, L.tm_gu, d.d, 2 * d.ffn, plan,
                          EpiSwigluArgs{static_cast<__half*>(c->h), d.ffn, L.s_gu, c->ssp, n_slots, inv_d, d.rms_eps},
-                         c->status, c->num_sms, s));
+                         c->status, c->gemm_grid, s));
       const bool last = l + 1 == n_layers;
       LCK(DUOLM_PROF_GEMM_DOWN,
           gemm_tc_resid(c->tm_h, L.tm_d, d.ffn, d.d, plan,
                         EpiResidArgs{c->x, d.d, L.s_d, last ? nullptr : xg,
                                      last ? nullptr : c->gains + c->layers[l + 1].g_attn, c->ssp, n_slots},
-                        c->status, c->num_sms, s));
+                        c->status, c->gemm_grid, s));
     }
   } else {
     float* xn = static_cast<float*>(c->xn);
@@ -475,6 +476,7 @@ int duolm_model_load(const duolm_model_desc* desc, const void* const* host_weigh
   if (cudaSetDevice(device) != cudaSuccess) return bail(DUOLM_E_CUDA);
   if (cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
     return bail(DUOLM_E_CUDA);
+  ctx->gemm_grid = ctx->num_sms & ~1;
   if (cuda_stream) {
     ctx->stream = static_cast<cudaStream_t>(cuda_stream);
   } else {
@@ -536,10 +538,11 @@ int duolm_model_load(const duolm_model_desc* desc, const void* const* host_weigh
       if ((rc = upload_f16(ctx, gu, D, &L.wgu, &L.s_gu, "w_gate/w_up"))) return bail(rc);
       if ((rc = upload_f16(ctx, {P(b + 10, D)}, F, &L.wd, &L.s_d, "w_down"))) return bail(rc);
       char e[256];
-      if (!make_tmap_f16_2d(&L.tm_qkv, L.wqkv, D, ctx->qd + 2 * ctx->kd, 64, 256, e, sizeof e) ||
-          !make_tmap_f16_2d(&L.tm_o, L.wo, ctx->qd, D, 64, 256, e, sizeof e) ||
-          !make_tmap_f16_2d(&L.tm_gu, L.wgu, D, 2 * F, 64, 256, e, sizeof e) ||
-          !make_tmap_f16_2d(&L.tm_d, L.wd, F, D, 64, 256, e, sizeof e)) {
+      // B tiles are loaded in halves of 128 rows, one per CTA of a pair
+      if (!make_tmap_f16_2d(&L.tm_qkv, L.wqkv, D, ctx->qd + 2 * ctx->kd, 64, 128, e, sizeof e) ||
+          !make_tmap_f16_2d(&L.tm_o, L.wo, ctx->qd, D, 64, 128, e, sizeof e) ||
+          !make_tmap_f16_2d(&L.tm_gu, L.wgu, D, 2 * F, 64, 128, e, sizeof e) ||
+          !make_tmap_f16_2d(&L.tm_d, L.wd, F, D, 64, 128, e, sizeof e)) {
         fail(ctx, DUOLM_E_CUDA, "%s", e);
         return bail(DUOLM_E_CUDA);
       }
@@ -958,7 +961,7 @@ int duolm_debug_gemm(duolm_ctx* ctx, int layer, int which, const uint16_t* a, fl
   if (e == cudaSuccess)
     e = gemm_tc_resid(ta, tb, K, N, reinterpret_cast<const PlanHdr*>(ctx->plan_dev),
                       EpiResidArgs{tmp, N, sc, nullptr, nullptr, nullptr, 0},
-                      ctx->status, ctx->num_sms, ctx->stream);
+                      ctx->status, ctx->gemm_grid, ctx->stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(out, tmp, T * N * 4, cudaMemcpyDeviceToHost, ctx->stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(ctx->stream);
   cudaFree(tmp);
