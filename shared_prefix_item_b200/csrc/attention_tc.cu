@@ -61,10 +61,8 @@ struct Item {
 };
 
 template <int G>
-__device__ __forceinline__ Item load_item(const PlanHdr* plan, int it, int b) {
+__device__ __forceinline__ Item make_item(int4 item, int4 rq, int b) {
   constexpr int R = kSlots / G;
-  const int4 item = plan_array<int4>(plan, plan->off_items)[it];
-  const int4 rq = plan_array<int4>(plan, plan->off_req)[item.x];
   Item m;
   m.tok0 = rq.x;
   m.L = rq.y;
@@ -79,6 +77,36 @@ __device__ __forceinline__ Item load_item(const PlanHdr* plan, int it, int b) {
   m.n_tiles = m.n_prefix_tiles + (m.branch ? 1 : 0);
   return m;
 }
+
+// Work-list reader that keeps the descriptors of the next two items in
+// flight, so a role never waits on global memory at an item boundary.
+template <int G>
+struct ItemStream {
+  const int4* items;
+  const int4* reqs;
+  int n, step, b;
+  int it;
+  int4 d1, d2, r1;  // descriptor of it + step, it + 2 step; request of it + step
+  __device__ ItemStream(const PlanHdr* plan, int first, int step_, int b_)
+      : items(plan_array<int4>(plan, plan->off_items)), reqs(plan_array<int4>(plan, plan->off_req)),
+        n(plan->n_items), step(step_), b(b_), it(first) {
+    const int4 z = make_int4(0, 0, 0, 0);
+    d1 = it < n ? items[it] : z;
+    d2 = it + step < n ? items[it + step] : z;
+    r1 = reqs[d1.x];
+  }
+  __device__ bool valid() const { return it < n; }
+  // the current item; advances the prefetch window
+  __device__ Item next() {
+    const Item m = make_item<G>(d1, r1, b);
+    const int4 z = make_int4(0, 0, 0, 0);
+    it += step;
+    d1 = d2;
+    r1 = reqs[d1.x];
+    d2 = it + step < n ? items[it + step] : z;
+    return m;
+  }
+};
 
 }  // namespace
 
@@ -96,7 +124,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (*reinterpret_cast<volatile const uint32_t*>(&st->flags) & ERR_WAIT_TIMEOUT) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_items = plan->n_items;
   const int b = plan->branch_len;
   constexpr int R = kSlots / G;
 
@@ -127,8 +154,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- TMA producer
     if (lane == 0) {
       uint32_t n_kv = 0, n_item = 0;
-      for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++n_item) {
-        const Item m = load_item<G>(plan, it, b);
+      for (ItemStream<G> is(plan, blockIdx.x, gridDim.x, b); is.valid(); ++n_item) {
+        const Item m = is.next();
         const uint32_t qs = n_item & 1, quse = n_item >> 1;
         if (!mbar_wait(bar(B_QEMPTY0 + qs), (quse & 1u) ^ 1u, st, 40)) break;
         mbar_arrive_expect_tx(bar(B_QFULL0 + qs), 2 * kHalf);
@@ -157,36 +184,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t n_kv = 0, n_s = 0, n_p = 0, n_item = 0;
       bool ok = true;
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++n_item) {
-        const Item m = load_item<G>(plan, it, b);
+      for (ItemStream<G> is(plan, blockIdx.x, gridDim.x, b); is.valid() && ok; ++n_item) {
+        const Item m = is.next();
         const uint32_t qs = n_item & 1, quse = n_item >> 1;
-        auto pv = [&](int t) -> bool {
-          if (!mbar_wait(bar(B_PFULL), (n_p + t) & 1u, st, 42)) return false;
-          tc_fence_after();
-          const uint32_t slot = (n_kv + t) & 1;
-#pragma unroll
-          for (int k = 0; k < kKeys / 16; ++k) {
-            const uint64_t da = smem_desc_sw128(sbase + kPOff + (k >> 2) * kHalf + (k & 3) * 32);
-            const uint64_t db = smem_desc_sw128_mn(sbase + kVOff + 2 * slot * kHalf + k * 2048, kHalf);
-            tc_mma_f16(tmemO, da, db, kIdescPV, (t > 0 || k > 0) ? 1u : 0u);
-          }
-          tc_commit(bar(B_KVEMPTY0 + slot));
-          tc_commit(bar(B_PEMPTY));
-          return true;
-        };
         if (!mbar_wait(bar(B_QFULL0 + qs), quse & 1u, st, 43)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        for (int t = 0; t < m.n_tiles && ok; ++t) {
-          const uint32_t slot = (n_kv + t) & 1, kuse = (n_kv + t) >> 1;
-          const uint32_t sb = (n_s + t) & 1, suse = (n_s + t) >> 1;
-          if (!mbar_wait(bar(B_KVFULL0 + slot), kuse & 1u, st, 44) ||
-              !mbar_wait(bar(B_SEMPTY0 + sb), (suse & 1u) ^ 1u, st, 45)) {
-            ok = false;
-            break;
-          }
+        // Issue S = QK^T of tile s_next and P V of tile pv_next in whatever
+        // order their inputs become ready (K/V tile landed and an S buffer
+        // free, or the softmax's P written), so neither waits on the other.
+        auto issue_s = [&](int t) {
+          const uint32_t slot = (n_kv + t) & 1;
+          const uint32_t sb = (n_s + t) & 1;
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < kHD / 16; ++k) {
@@ -196,9 +207,45 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_commit(bar(B_SFULL0 + sb));
           if (t == m.n_tiles - 1) tc_commit(bar(B_QEMPTY0 + qs));  // Q slot free once these S are done
-          if (t > 0 && !pv(t - 1)) ok = false;
+        };
+        auto issue_pv = [&](int t) {
+          const uint32_t slot = (n_kv + t) & 1;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < kKeys / 16; ++k) {
+            const uint64_t da = smem_desc_sw128(sbase + kPOff + (k >> 2) * kHalf + (k & 3) * 32);
+            const uint64_t db = smem_desc_sw128_mn(sbase + kVOff + 2 * slot * kHalf + k * 2048, kHalf);
+            tc_mma_f16(tmemO, da, db, kIdescPV, (t > 0 || k > 0) ? 1u : 0u);
+          }
+          tc_commit(bar(B_KVEMPTY0 + slot));
+          tc_commit(bar(B_PEMPTY));
+        };
+        int s_next = 0, pv_next = 0;
+        const uint64_t t0 = global_ns();
+        uint32_t spins = 0;
+        while (pv_next < m.n_tiles) {
+          bool progressed = false;
+          // S of the next tile: its K/V landed and its S buffer is free (the
+          // softmax is done with the tile two back); never more than one S
+          // ahead of the oldest P V not yet issued
+          if (s_next < m.n_tiles && s_next <= pv_next + 1) {
+            const uint32_t kuse = (n_kv + s_next) >> 1, suse = (n_s + s_next) >> 1;
+            if (mbar_try_wait(bar(B_KVFULL0 + ((n_kv + s_next) & 1)), kuse & 1u) &&
+                mbar_try_wait(bar(B_SEMPTY0 + ((n_s + s_next) & 1)), (suse & 1u) ^ 1u)) {
+              issue_s(s_next++);
+              progressed = true;
+            }
+          }
+          if (pv_next < s_next && mbar_try_wait(bar(B_PFULL), (n_p + pv_next) & 1u)) {
+            issue_pv(pv_next++);
+            progressed = true;
+          }
+          if (!progressed && (++spins & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) {
+            raise_error(st, ERR_WAIT_TIMEOUT, 44);
+            ok = false;
+            break;
+          }
         }
-        if (ok && !pv(m.n_tiles - 1)) ok = false;
         if (ok) tc_commit(bar(B_OFULL));
         n_kv += m.n_tiles;
         n_s += m.n_tiles;
@@ -232,8 +279,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     uint32_t n_s = 0, n_p = 0, n_item = 0;
     bool ok = true;
-    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++n_item) {
-      const Item m = load_item<G>(plan, it, b);
+    for (ItemStream<G> is(plan, blockIdx.x, gridDim.x, b); is.valid() && ok; ++n_item) {
+      const Item m = is.next();
       const KeyRange kr = tree_keys(m.q0 + r / G, m.L, b);
       float m_used = -INFINITY, l = 0.f;
       for (int t = 0; t < m.n_tiles && ok; ++t) {

@@ -730,27 +730,34 @@ int duolm_prepare(duolm_ctx* ctx, int n_requests, const int32_t* prefix_ids, con
       cand[c++] = (int32_t)(t - 1);  // the branch's last token is scored
     }
   }
-  // attention work items, most expensive first (fp16 path)
+  // attention work items (fp16 path).  The items of one (request, KV head)
+  // stay together so that the CTAs running them at the same time share that
+  // head's prefix K/V through L2; groups go most expensive first, and inside
+  // a group branch items come first, then prefix items from the last rows.
   int64_t n_items = 0;
   if (ctx->f16) {
     const int Rw = ctx->rows_per_item;
     const int per = (Rw / branch_len) * branch_len;
-    std::vector<std::pair<int, int4>> items;
-    items.reserve(ctx->cap_I);
+    const int key_tile = 128;
+    std::vector<std::pair<int64_t, int64_t>> groups;  // (cost in key tiles, request * n_kv_heads + kvh)
+    groups.reserve((size_t)R * ctx->desc.n_kv_heads);
     for (int64_t r = 0; r < R; ++r) {
       const int L = rq[r].y, K = rq[r].z;
-      for (int kvh = 0; kvh < ctx->desc.n_kv_heads; ++kvh) {
-        for (int row0 = 0; row0 < L; row0 += Rw)
-          items.push_back({(std::min(row0 + Rw, L) + 63) / 64, int4{(int)r, kvh, 0, row0}});
-        for (int row0 = 0; row0 < K * branch_len; row0 += per)
-          items.push_back({(L + 63) / 64 + 1, int4{(int)r, kvh, 1, row0}});
-      }
+      int64_t cost = 0;
+      for (int row0 = 0; row0 < L; row0 += Rw) cost += (std::min(row0 + Rw, L) + key_tile - 1) / key_tile;
+      cost += (int64_t)((K * branch_len + per - 1) / per) * ((L + key_tile - 1) / key_tile + 1);
+      for (int kvh = 0; kvh < ctx->desc.n_kv_heads; ++kvh) groups.push_back({cost, r * ctx->desc.n_kv_heads + kvh});
     }
-    if ((int64_t)items.size() > ctx->cap_I) return fail(ctx, DUOLM_E_CAPACITY, "prepare: work list overflow");
-    std::stable_sort(items.begin(), items.end(), [](const auto& a, const auto& b) { return a.first > b.first; });
+    std::stable_sort(groups.begin(), groups.end(), [](const auto& a, const auto& b) { return a.first > b.first; });
     int4* it = reinterpret_cast<int4*>(base + hdr.off_items);
-    for (size_t i = 0; i < items.size(); ++i) it[i] = items[i].second;
-    n_items = (int64_t)items.size();
+    for (const auto& g : groups) {
+      const int r = (int)(g.second / ctx->desc.n_kv_heads), kvh = (int)(g.second % ctx->desc.n_kv_heads);
+      const int L = rq[r].y, K = rq[r].z;
+      const int64_t need = (K * branch_len + per - 1) / per + (L + Rw - 1) / Rw;
+      if (n_items + need > ctx->cap_I) return fail(ctx, DUOLM_E_CAPACITY, "prepare: work list overflow");
+      for (int row0 = 0; row0 < K * branch_len; row0 += per) it[n_items++] = int4{r, kvh, 1, row0};
+      for (int row0 = ((L - 1) / Rw) * Rw; row0 >= 0; row0 -= Rw) it[n_items++] = int4{r, kvh, 0, row0};
+    }
   }
   hdr.n_items = (int32_t)n_items;
   const int64_t bytes = hdr.off_items + align16(n_items * 16);
