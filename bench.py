@@ -53,6 +53,19 @@ def workload(name: str, shard: int) -> W.Workload:
     raise SystemExit(f"unknown config {name}")
 
 
+def combine_ranks(dist, ms: float, units: int, device) -> tuple:
+    """Whole-job figures from one rank's own: the slowest rank's time (every
+    rank scores its own shard, so the job ends when the last one does) and
+    the units scored by all ranks together.  ``dist`` is None on one rank."""
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    u = torch.tensor([units], dtype=torch.int64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), int(u.item())
+
+
 def describe(wl: W.Workload, mode: str, graph: bool, n: int) -> dict:
     Ls = [r.L for r in wl.requests]
     return {
@@ -297,11 +310,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         barrier()
     rk.sync()
     ms = start.elapsed_time(end) / args.steps
-    ms_t = torch.tensor([ms], device="cuda")
-    if dist:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
-    value = n_cand * world / (ms_max / 1e3)
+    ms_max, n_total = combine_ranks(dist, ms, n_cand, "cuda")
+    value = n_total / (ms_max / 1e3)
     launches = rk.launches_per_execute()
 
     # e2e: the public call from host buffers, scores back to the host every step
@@ -315,10 +325,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     end.record(stream)
     barrier()
     e2e_ms = start.elapsed_time(end) / args.steps
-    e2e_t = torch.tensor([e2e_ms], device="cuda")
-    if dist:
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-    e2e_value = n_cand * world / (float(e2e_t.item()) / 1e3)
+    e2e_max, _ = combine_ranks(dist, e2e_ms, n_cand, "cuda")
+    e2e_value = n_total / (e2e_max / 1e3)
 
     # per-kernel-class device time (eager launches with an event after each)
     rk.prepare(p, po, b, co, wl.branch_len, mode)

@@ -26,6 +26,9 @@ struct DevStatus {
 };
 
 __device__ __forceinline__ void raise_error(DevStatus* st, uint32_t flag, uint32_t where) {
+  // a plain read first: once the flag is up, further reports (possibly one
+  // per element of a bad tensor) do not queue atomics on one word
+  if (*reinterpret_cast<volatile uint32_t*>(&st->flags) & flag) return;
   uint32_t old = atomicOr(&st->flags, flag);
   if (old == 0) st->where = where;
 }
