@@ -3,29 +3,38 @@
 // DuoLM summary page (paper.rainbus.top), 方法步骤详情 step 4 and 研究动机:
 // the prefix of a request is computed once and its K/V are shared by all K
 // candidate branches; candidate j attends to the prefix and to its own branch
-// only.  Work is cut into items of 128 query slots of one request and one KV
-// head (a slot is a (token, query head of the KV head's group) pair; 64
-// tokens x 2 heads for Qwen3's grouping):
-//   kind 0  prefix tokens [row0, row0 + R): causal over the prefix;
-//   kind 1  branch tokens [row0, row0 + R') (whole candidates): every prefix
-//           key, then one extra 128-key tile of branch rows under the tree rule.
-// Per item each KV head's prefix tiles stream through shared memory once for
-// all 128 slots.  One CTA per SM, 320 threads:
-//   warp 0   TMA: Q (3-D map, 2 x 16 KB, double buffered so the next item's
-//            Q arrives early), then K and V tiles of 128 keys (2 x 32 KB
-//            each, double buffered); 128-byte swizzle, no multicast;
-//   warp 1   one lane issues tcgen05.mma: S = Q K^T (M 128, N 128 keys,
-//            K-major operands) into one of two TMEM S buffers, then
-//            O += P V (P from shared memory K-major, V MN-major) into TMEM;
-//            S of tile t + 1 is issued before P V of tile t;
-//   warps 2-9 softmax, two threads per slot row (TMEM lane), each on half of
-//            the keys: load S, mask, row max (halves combined through shared
-//            memory), P = 2^(s - m) in fp16 to shared memory, row sum; O in
-//            TMEM is rescaled only when the running max grows by more than
-//            2^8 (P stays below 256, exact after the final division);
-//            finally O / l to global memory.
-// The three roles run ahead of each other across item boundaries; every
-// mbarrier wait is bounded, and after a timeout the kernel raises the status
+// only.  Work is cut into items of one request and one KV head.  An item holds
+// two sub-tiles A and B of 128 query slots each (a slot is a (token, query
+// head of the KV head's group) pair: 64 tokens x 2 heads per sub-tile for
+// Qwen3's grouping), and every K/V tile the item loads serves both:
+//   kind 0  prefix tokens [row0, row0 + 2R): causal over the prefix;
+//   kind 1  branch tokens (whole candidates): every prefix key tile, then the
+//           tiles of the item's own branch rows under the tree rule.
+// B is left out when the item's rows all fit in A.  One CTA per SM, 384
+// threads in three warpgroups:
+//   warps 0-3 softmax of A, warps 4-7 softmax of B: one thread per slot row
+//             (TMEM lane) and 128 keys: load S, mask, row max, P = 2^(s - m)
+//             as fp16 written back over S in tensor memory, row sum; O_X is
+//             rescaled only when the running max grows by more than 2^8 (P
+//             stays below 256, exact after the final division); at the end of
+//             an item O_X / l to global memory;
+//   warp 8    TMA: Q of A and B (3-D map, 32 KB each), K and V tiles of 128
+//             keys (32 KB each, two slots each, separate barriers so a K tile
+//             can land while the previous V is still in use); 128-byte
+//             swizzle, no multicast;
+//   warp 9    one lane issues tcgen05.mma, per key tile and per sub-tile X:
+//             O_X (+)= P_X V of the previous tile (P read from tensor
+//             memory), then S_X = Q_X K^T of this tile into the same columns;
+//   warps 10-11 idle.
+// The softmax warpgroups hold a whole 128-key row of S in registers: they
+// take registers from the third warpgroup (setmaxnreg; 2 x 128 x kRegSoftmax
+// + 128 x kRegOther is exactly the launch's 384 x 168).
+// Tensor memory: S/P of A in columns [0, 128), of B in [128, 256), O of A in
+// [256, 384), O of B in [384, 512).  tcgen05.mma operations issued by one
+// thread run in issue order, so S_X of a tile may be issued right after the
+// P V that reads the same columns, and the commit that reports S_X complete
+// also reports the preceding P V complete (O_X current for a rescale).
+// Every mbarrier wait is bounded; after a timeout the kernel raises the status
 // flag and returns.
 #include "common.cuh"
 #include "kernels.cuh"
@@ -34,35 +43,41 @@ namespace duolm {
 
 namespace {
 
-constexpr int kSlots = 128;   // query slots per item (MMA M)
-constexpr int kKeys = 128;    // keys per tile (MMA N of Q K^T)
+constexpr int kSub = 128;   // query slots per sub-tile (MMA M)
+constexpr int kKeys = 128;  // keys per tile (MMA N of Q K^T)
 constexpr int kHD = 128;
-constexpr int kSoftmax = 256;             // 8 softmax warps: two per TMEM lane quadrant
-constexpr int kThreads = 64 + kSoftmax;
-constexpr int kHalf = 16384;  // one 128-row x 64-element fp16 box
-constexpr int kQOff = 0;                  // Q: 2 slots x 2 boxes (next item's Q loads early)
-constexpr int kKOff = 4 * kHalf;          // K: 2 slots x 2 boxes
-constexpr int kVOff = kKOff + 4 * kHalf;  // V: 2 slots x 2 boxes
-constexpr int kPOff = kVOff + 4 * kHalf;  // P: 2 boxes
-constexpr int kBarOff = kPOff + 2 * kHalf;
-constexpr int kRedOff = kBarOff + 256;     // per-row partial maxima / sums of the two column halves
-constexpr int kSmem = kRedOff + 2 * 128 * 4 + 1024;
-constexpr uint32_t kIdescS = idesc_f16_f32(128, kKeys);
-constexpr uint32_t kIdescPV = idesc_f16_f32_bmn(128, kHD);
-constexpr uint32_t kTmemCols = 512;  // S0 [0,128), S1 [128,256), O [256,384)
+constexpr int kSoftmaxWG = 128;  // threads of one softmax warpgroup
+constexpr int kThreads = 3 * kSoftmaxWG;
+constexpr int kWarpTma = 8, kWarpMma = 9;
+constexpr int kRegLaunch = 168;  // 65536 / 384 rounded down to a multiple of 8
+constexpr int kRegSoftmax = 200, kRegOther = 104;
+static_assert(2 * kSoftmaxWG * kRegSoftmax + kSoftmaxWG * kRegOther <= kThreads * kRegLaunch,
+              "register split above the launch's registers");
+constexpr int kHalf = 16384;         // one 128-row x 64-element fp16 box
+constexpr int kQOff = 0;             // Q: 2 sub-tiles x 2 boxes
+constexpr int kKOff = 4 * kHalf;     // K: 2 slots x 2 boxes
+constexpr int kVOff = 8 * kHalf;     // V: 2 slots x 2 boxes
+constexpr int kBarOff = 12 * kHalf;
+constexpr int kSmem = kBarOff + 256 + 1024;
+constexpr uint32_t kIdescS = idesc_f16_f32(kSub, kKeys);
+constexpr uint32_t kIdescPV = idesc_f16_f32_bmn(kSub, kHD);
+constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 
-enum { B_QFULL0, B_QFULL1, B_QEMPTY0, B_QEMPTY1, B_KVFULL0, B_KVFULL1, B_KVEMPTY0, B_KVEMPTY1, B_SFULL0,
-       B_SFULL1, B_SEMPTY0, B_SEMPTY1, B_PFULL, B_PEMPTY, B_OFULL, B_DRAIN, B_COUNT };
+enum { B_QFULL0, B_QFULL1, B_QEMPTY0, B_QEMPTY1, B_KFULL0, B_KFULL1, B_VFULL0, B_VFULL1, B_KEMPTY0, B_KEMPTY1,
+       B_VEMPTY0, B_VEMPTY1, B_SFULL0, B_SFULL1, B_PFULL0, B_PFULL1, B_OFULL0, B_OFULL1, B_DRAIN, B_COUNT };
 
 struct Item {
-  int tok0, L, K, kvh, branch, row0, q0, nrows, n_prefix_tiles, n_tiles;
-  __device__ int tile_start(int t) const { return t < n_prefix_tiles ? t * kKeys : q0; }
+  int tok0, L, K, kvh, branch, row0, q0, nrows, n_prefix_tiles, n_tiles, has_b;
+  __device__ int tile_start(int t) const {
+    return t < n_prefix_tiles ? t * kKeys : q0 + (t - n_prefix_tiles) * kKeys;
+  }
 };
 
 template <int G>
 __device__ __forceinline__ Item make_item(int4 item, int4 rq, int b) {
-  constexpr int R = kSlots / G;
+  constexpr int R = kSub / G;  // tokens per sub-tile
+  constexpr int R2 = 2 * R;    // tokens per item
   Item m;
   m.tok0 = rq.x;
   m.L = rq.y;
@@ -71,10 +86,11 @@ __device__ __forceinline__ Item make_item(int4 item, int4 rq, int b) {
   m.branch = item.z;
   m.row0 = item.w;
   m.q0 = m.branch ? m.L + m.row0 : m.row0;
-  m.nrows = m.branch ? min((R / b) * b, m.K * b - m.row0) : min(R, m.L - m.row0);
-  const int kend = m.branch ? m.L : min(m.row0 + R, m.L);
+  m.nrows = m.branch ? min((R2 / b) * b, m.K * b - m.row0) : min(R2, m.L - m.row0);
+  const int kend = m.branch ? m.L : min(m.row0 + R2, m.L);
   m.n_prefix_tiles = (kend + kKeys - 1) / kKeys;
-  m.n_tiles = m.n_prefix_tiles + (m.branch ? 1 : 0);
+  m.n_tiles = m.n_prefix_tiles + (m.branch ? (m.nrows + kKeys - 1) / kKeys : 0);
+  m.has_b = m.nrows > R;
   return m;
 }
 
@@ -125,19 +141,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (*reinterpret_cast<volatile const uint32_t*>(&st->flags) & ERR_WAIT_TIMEOUT) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = plan->branch_len;
-  constexpr int R = kSlots / G;
+  constexpr int R = kSub / G;
 
-  if (warp == 0 && lane == 0) {
+  if (warp == kWarpTma && lane == 0) {
     prefetch_tensormap(&tmQ);
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
-    for (int i = 0; i < B_COUNT; ++i) {
-      const uint32_t cnt = (i == B_SEMPTY0 || i == B_SEMPTY1 || i == B_PFULL) ? (uint32_t)kSoftmax : 1u;
-      mbar_init(bar(i), cnt);
-    }
+    for (int i = 0; i < B_COUNT; ++i)
+      mbar_init(bar(i), (i == B_PFULL0 || i == B_PFULL1) ? (uint32_t)kSoftmaxWG : 1u);
     fence_barrier_init();
   }
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tmem_alloc(smem_u32(tmem_holder), kTmemCols);
     tmem_relinquish();
   }
@@ -145,285 +159,267 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tmemO = tmem + 256;
 
   // Every role walks the same items and tiles, so the running counts below
-  // (items, KV tiles, S buffers, P buffers) agree across roles and give each
-  // barrier's phase.  Roles run ahead of each other across item boundaries.
-  if (warp == 0) {
-    // ---- TMA producer
-    if (lane == 0) {
-      uint32_t n_kv = 0, n_item = 0;
-      for (ItemStream<G> is(plan, blockIdx.x, gridDim.x, b); is.valid(); ++n_item) {
-        const Item m = is.next();
-        const uint32_t qs = n_item & 1, quse = n_item >> 1;
-        if (!mbar_wait(bar(B_QEMPTY0 + qs), (quse & 1u) ^ 1u, st, 40)) break;
-        mbar_arrive_expect_tx(bar(B_QFULL0 + qs), 2 * kHalf);
-        for (int h = 0; h < 2; ++h)
-          tma_load_3d(&tmQ, sbase + kQOff + (2 * qs + h) * kHalf, bar(B_QFULL0 + qs), h * 64, m.kvh * G,
-                      m.tok0 + m.q0);
-        bool ok = true;
-        for (int t = 0; t < m.n_tiles; ++t, ++n_kv) {
-          const uint32_t slot = n_kv & 1, use = n_kv >> 1;
-          if (!mbar_wait(bar(B_KVEMPTY0 + slot), (use & 1u) ^ 1u, st, 41)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(bar(B_KVFULL0 + slot), 4 * kHalf);
-          const int y = (int)((int64_t)m.kvh * kv_rows + m.tok0 + m.tile_start(t));
-          for (int h = 0; h < 2; ++h) {
-            tma_load_2d(&tmK, sbase + kKOff + (2 * slot + h) * kHalf, bar(B_KVFULL0 + slot), h * 64, y);
-            tma_load_2d(&tmV, sbase + kVOff + (2 * slot + h) * kHalf, bar(B_KVFULL0 + slot), h * 64, y);
-          }
-        }
-        if (!ok) break;
-      }
-    }
-  } else if (warp == 1) {
-    // ---- MMA issuer
-    if (lane == 0) {
-      uint32_t n_kv = 0, n_s = 0, n_p = 0, n_item = 0;
-      bool ok = true;
-      for (ItemStream<G> is(plan, blockIdx.x, gridDim.x, b); is.valid() && ok; ++n_item) {
-        const Item m = is.next();
-        const uint32_t qs = n_item & 1, quse = n_item >> 1;
-        if (!mbar_wait(bar(B_QFULL0 + qs), quse & 1u, st, 43)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // Issue S = QK^T of tile s_next and P V of tile pv_next in whatever
-        // order their inputs become ready (K/V tile landed and an S buffer
-        // free, or the softmax's P written), so neither waits on the other.
-        auto issue_s = [&](int t) {
-          const uint32_t slot = (n_kv + t) & 1;
-          const uint32_t sb = (n_s + t) & 1;
-          tc_fence_after();
-#pragma unroll
-          for (int k = 0; k < kHD / 16; ++k) {
-            const uint64_t da = smem_desc_sw128(sbase + kQOff + (2 * qs + (k >> 2)) * kHalf + (k & 3) * 32);
-            const uint64_t db = smem_desc_sw128(sbase + kKOff + (2 * slot + (k >> 2)) * kHalf + (k & 3) * 32);
-            tc_mma_f16(tmem + sb * kKeys, da, db, kIdescS, k > 0 ? 1u : 0u);
-          }
-          tc_commit(bar(B_SFULL0 + sb));
-          if (t == m.n_tiles - 1) tc_commit(bar(B_QEMPTY0 + qs));  // Q slot free once these S are done
-        };
-        auto issue_pv = [&](int t) {
-          const uint32_t slot = (n_kv + t) & 1;
-          tc_fence_after();
-#pragma unroll
-          for (int k = 0; k < kKeys / 16; ++k) {
-            const uint64_t da = smem_desc_sw128(sbase + kPOff + (k >> 2) * kHalf + (k & 3) * 32);
-            const uint64_t db = smem_desc_sw128_mn(sbase + kVOff + 2 * slot * kHalf + k * 2048, kHalf);
-            tc_mma_f16(tmemO, da, db, kIdescPV, (t > 0 || k > 0) ? 1u : 0u);
-          }
-          tc_commit(bar(B_KVEMPTY0 + slot));
-          tc_commit(bar(B_PEMPTY));
-        };
-        int s_next = 0, pv_next = 0;
-        const uint64_t t0 = global_ns();
-        uint32_t spins = 0;
-        while (pv_next < m.n_tiles) {
-          bool progressed = false;
-          // S of the next tile: its K/V landed and its S buffer is free (the
-          // softmax is done with the tile two back); never more than one S
-          // ahead of the oldest P V not yet issued
-          if (s_next < m.n_tiles && s_next <= pv_next + 1) {
-            const uint32_t kuse = (n_kv + s_next) >> 1, suse = (n_s + s_next) >> 1;
-            if (mbar_try_wait(bar(B_KVFULL0 + ((n_kv + s_next) & 1)), kuse & 1u) &&
-                mbar_try_wait(bar(B_SEMPTY0 + ((n_s + s_next) & 1)), (suse & 1u) ^ 1u)) {
-              issue_s(s_next++);
-              progressed = true;
-            }
-          }
-          if (pv_next < s_next && mbar_try_wait(bar(B_PFULL), (n_p + pv_next) & 1u)) {
-            issue_pv(pv_next++);
-            progressed = true;
-          }
-          if (!progressed && (++spins & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) {
-            raise_error(st, ERR_WAIT_TIMEOUT, 44);
-            ok = false;
-            break;
-          }
-        }
-        if (ok) tc_commit(bar(B_OFULL));
-        n_kv += m.n_tiles;
-        n_s += m.n_tiles;
-        n_p += m.n_tiles;
-      }
-      // no tensor-core operation of this CTA may outlive its TMEM
-      tc_commit(bar(B_DRAIN));
-      mbar_wait(bar(B_DRAIN), 0, st, 46);
-    }
-  } else {
-    // ---- softmax: thread = (slot row r = TMEM lane, column half ch); the two
-    // threads of a row exchange partial maxima (and at the end the sums)
-    // through shared memory
+  // (K/V tiles, and per sub-tile its items and tiles) agree across roles and
+  // give each barrier's phase.
+  if (warp < 8) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegSoftmax));
+    // ---- softmax of sub-tile X: thread = slot row r = TMEM lane
+    const int X = warp >> 2;
     const int q4 = warp & 3;
-    const int ch = (warp - 2) >> 2;  // 0: keys / dims [0, 64), 1: [64, 128)
     const int r = q4 * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    float* red = reinterpret_cast<float*>(smem + kRedOff);  // [2][128]
-    // Barrier over the softmax threads that also ANDs a flag across them, so
-    // that a failed (timed-out) wait stops all eight warps together and none
-    // is left at a named barrier.
-    auto softmax_all = [](bool v) -> bool {
-      uint32_t res;
-      asm volatile(
-          "{ .reg .pred pin, pout; setp.ne.u32 pin, %1, 0; bar.red.and.pred pout, 1, %2, pin; "
-          "selp.u32 %0, 1, 0, pout; }"
-          : "=r"(res)
-          : "r"(v ? 1u : 0u), "n"(kSoftmax)
-          : "memory");
-      return res != 0;
-    };
-    uint32_t n_s = 0, n_p = 0, n_item = 0;
+    const uint32_t tS = tmem + lane_off + 128 * X, tO = tmem + lane_off + 256 + 128 * X;
+    uint32_t n_xt = 0, n_xi = 0;
     bool ok = true;
-    for (ItemStream<G> is(plan, blockIdx.x, gridDim.x, b); is.valid() && ok; ++n_item) {
+    for (ItemStream<G> is(plan, blockIdx.x, gridDim.x, b); is.valid() && ok;) {
       const Item m = is.next();
-      const KeyRange kr = tree_keys(m.q0 + r / G, m.L, b);
+      if (X == 1 && !m.has_b) continue;
+      const int rl = X * R + r / G;  // row of the item (token offset from q0)
+      const KeyRange kr = tree_keys(m.q0 + rl, m.L, b);
       float m_used = -INFINITY, l = 0.f;
-      for (int t = 0; t < m.n_tiles && ok; ++t) {
-        const uint32_t sb = (n_s + t) & 1, suse = (n_s + t) >> 1;
-        if (!softmax_all(mbar_wait_warp(bar(B_SFULL0 + sb), suse & 1u, st, 47))) {
+      for (int t = 0; t < m.n_tiles; ++t, ++n_xt) {
+        if (!mbar_wait_warp(bar(B_SFULL0 + X), n_xt & 1u, st, 48)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const int k0 = m.tile_start(t) + 64 * ch;
-        const bool is_branch_tile = m.branch && t == m.n_prefix_tiles;
-        const bool need_mask = is_branch_tile || (!m.branch && m.tile_start(t) + kKeys > m.row0) ||
-                               (m.branch && m.tile_start(t) + kKeys > m.L);
-        const uint32_t s_addr = tmem + lane_off + sb * kKeys + 64 * ch;
-        // this thread's 64 S values: two loads, one wait
-        uint32_t sr[2][32];
+        uint32_t sr[4][32];
 #pragma unroll
-        for (int q = 0; q < 2; ++q) tmem_ld32_async(s_addr + 32 * q, sr[q]);
+        for (int c = 0; c < 4; ++c) tmem_ld32_async(tS + 32 * c, sr[c]);
         tmem_wait_ld();
-        float mx = -INFINITY;
 #pragma unroll
-        for (int q = 0; q < 2; ++q)
+        for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            tmem_ld_fence(sr[q][j]);
-            float x = __uint_as_float(sr[q][j]) * scale_log2;
-            if (need_mask) {
-              const int tk = k0 + 32 * q + j;
-              const bool vis = is_branch_tile ? (tk >= kr.br_lo && tk <= kr.br_hi) : (tk <= kr.pre_hi);
-              if (!vis) x = -INFINITY;
-            }
-            sr[q][j] = __float_as_uint(x);
-            mx = fmaxf(mx, x);
-          }
-        // S buffer consumed: the MMA may refill it
-        tc_fence_before();
-        mbar_arrive(bar(B_SEMPTY0 + sb));
-        // row max over both halves; the barrier that publishes the partial
-        // maxima also confirms the P buffer is free and O complete for the
-        // previous tile (the next tile's writes of red[] come after its first
-        // barrier, which every thread reaches only after reading red[] here)
-        red[ch * 128 + r] = mx;
-        if (!softmax_all(mbar_wait_warp(bar(B_PEMPTY), ((n_p + t) & 1u) ^ 1u, st, 48))) {
-          ok = false;
-          break;
+          for (int j = 0; j < 32; ++j) tmem_ld_fence(sr[c][j]);
+        const int k0 = m.tile_start(t);
+        const bool is_branch_tile = t >= m.n_prefix_tiles;
+        const bool need_mask = is_branch_tile || (!m.branch && k0 + kKeys > m.row0) || (m.branch && k0 + kKeys > m.L);
+        if (need_mask) {
+          // this row's visible keys in the tile are one window [lo0, lo0 + n)
+          // of tile-local indices: its own branch keys in a branch tile, the
+          // prefix keys up to pre_hi otherwise
+          const int lo = is_branch_tile ? kr.br_lo - k0 : 0;
+          const int hi = is_branch_tile ? kr.br_hi - k0 : kr.pre_hi - k0;  // inclusive
+          const uint32_t lo0 = (uint32_t)max(lo, 0);
+          const uint32_t n = (uint32_t)max(0, min(hi, kKeys - 1) - max(lo, 0) + 1);
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if ((uint32_t)(32 * c + j) - lo0 >= n) sr[c][j] = __float_as_uint(-INFINITY);
         }
-        mx = fmaxf(mx, red[(ch ^ 1) * 128 + r]);
-        tc_fence_after();
-        const float m_new = fmaxf(m_used, mx);
+        // row max of the raw scores (the scale is positive: applied after)
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) mx[j & 3] = fmaxf(mx[j & 3], __uint_as_float(sr[c][j]));
+        const float m_new = fmaxf(m_used, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * scale_log2);
         // the O rescale uses warp-collective TMEM loads and stores: decide it
-        // for the whole warp (both warps of a row group see the same maxima,
-        // so they decide alike; a row that did not need it is rescaled to its
+        // for the whole warp (a row that did not need it is rescaled to its
         // new max as well, which is just as exact)
         if (t == 0) {
           m_used = m_new;
         } else if (__any_sync(0xffffffffu, m_new > m_used + kRescaleLog2)) {
           const float corr = m_new == m_used ? 1.f : fast_exp2(m_used - m_new);  // 0 while nothing was visible
 #pragma unroll 1
-          for (int c = 64 * ch; c < 64 * ch + 64; c += 32) {
+          for (int c = 0; c < 4; ++c) {
             float v[32];
-            tmem_ld32(tmemO + lane_off + c, v);
+            tmem_ld32(tO + 32 * c, v);
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] *= corr;
-            tmem_st32(tmemO + lane_off + c, v);
+            tmem_st32(tO + 32 * c, v);
           }
           l *= corr;
           m_used = m_new;
         }
-        const float mu = m_used == -INFINITY ? 0.f : m_used;
-        // P = 2^(s - mu) in fp16 into this half's K-major 128-byte-swizzled box
-        float sum = 0.f;
-        const uint32_t pbox = sbase + kPOff + ch * kHalf + (r >> 3) * 1024 + (r & 7) * 128;
+        const float nmu = m_used == -INFINITY ? 0.f : -m_used;
+        // P = 2^(s scale - m) in fp16 over the first 64 columns of S
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
-            const float p0 = fast_exp2(__uint_as_float(sr[q][j]) - mu);
-            const float p1 = fast_exp2(__uint_as_float(sr[q][j + 1]) - mu);
-            sum += p0 + p1;
-            const __half2 h = __floats2half2_rn(p0, p1);
-            pk[j / 2] = *reinterpret_cast<const uint32_t*>(&h);
+            const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c][j]), scale_log2, nmu));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c][j + 1]), scale_log2, nmu));
+            ls[(j >> 1) & 3] += p0 + p1;
+            pk[j / 2] = pack_half2(p0, p1);
           }
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int chunk = q * 4 + u;
-            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(pbox + ((chunk ^ (r & 7)) << 4)),
-                         "r"(pk[4 * u]), "r"(pk[4 * u + 1]), "r"(pk[4 * u + 2]), "r"(pk[4 * u + 3])
-                         : "memory");
-          }
+          tmem_st16_async(tS + 16 * c, pk);
         }
-        l += sum;
+        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        tmem_wait_st();
         tc_fence_before();
-        fence_proxy_async_smem();
-        mbar_arrive(bar(B_PFULL));
+        mbar_arrive(bar(B_PFULL0 + X));
       }
-      // ---- epilogue: O / l -> fp16, this thread's 64 dims (O is
-      // overwritten only after the next item's first P, which these warps
-      // release after this read)
       if (!ok) break;
-      // (this barrier also orders the partner's read of the last partial
-      // max before the sum overwrites it)
-      if (!softmax_all(mbar_wait_warp(bar(B_OFULL), n_item & 1u, st, 49))) {
+      // ---- end of the item: O_X / l -> fp16, this thread's row (O_X is
+      // overwritten only by the P V of the next item's first P, which this
+      // thread releases after this read)
+      if (!mbar_wait_warp(bar(B_OFULL0 + X), n_xi & 1u, st, 49)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      red[ch * 128 + r] = l;
-      asm volatile("bar.sync 1, %0;" ::"n"(kSoftmax) : "memory");
-      l += red[(ch ^ 1) * 128 + r];
+      ++n_xi;
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      const int rl = r / G;
       const bool valid = rl < m.nrows;
       __half* dst = o + (((int64_t)m.tok0 + m.q0 + rl) * n_q_heads + m.kvh * G + (r % G)) * kHD;
 #pragma unroll 1
-      for (int c = 64 * ch; c < 64 * ch + 64; c += 32) {
+      for (int c = 0; c < 4; ++c) {
         float v[32];
-        tmem_ld32(tmemO + lane_off + c, v);
+        tmem_ld32(tO + 32 * c, v);
         if (valid) {
-          uint32_t pk[16];
+          uint32_t pw[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const __half2 h = __floats2half2_rn(v[2 * j] * inv, v[2 * j + 1] * inv);
-            pk[j] = *reinterpret_cast<const uint32_t*>(&h);
-          }
-          uint4* p = reinterpret_cast<uint4*>(dst + c);
+          for (int j = 0; j < 16; ++j) pw[j] = pack_half2(v[2 * j] * inv, v[2 * j + 1] * inv);
+          uint4* p = reinterpret_cast<uint4*>(dst + 32 * c);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) p[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          for (int q = 0; q < 4; ++q) p[q] = make_uint4(pw[4 * q], pw[4 * q + 1], pw[4 * q + 2], pw[4 * q + 3]);
         }
       }
       tc_fence_before();
-      n_s += m.n_tiles;
-      n_p += m.n_tiles;
+    }
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegOther));
+    if (warp == kWarpTma) {
+      // ---- TMA producer
+      if (lane == 0) {
+        uint32_t n_kv = 0, n_xi[2] = {0, 0};
+        bool ok = true;
+        for (ItemStream<G> is(plan, blockIdx.x, gridDim.x, b); is.valid() && ok;) {
+          const Item m = is.next();
+#pragma unroll
+          for (int X = 0; X < 2; ++X) {
+            if (X > m.has_b) break;
+            if (!mbar_wait(bar(B_QEMPTY0 + X), (n_xi[X] & 1u) ^ 1u, st, 40)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(bar(B_QFULL0 + X), 2 * kHalf);
+            for (int h = 0; h < 2; ++h)
+              tma_load_3d(&tmQ, sbase + kQOff + (2 * X + h) * kHalf, bar(B_QFULL0 + X), h * 64, m.kvh * G,
+                          m.tok0 + m.q0 + X * R);
+            ++n_xi[X];
+          }
+          for (int t = 0; t < m.n_tiles && ok; ++t, ++n_kv) {
+            const uint32_t slot = n_kv & 1, use = n_kv >> 1;
+            const int y = (int)((int64_t)m.kvh * kv_rows + m.tok0 + m.tile_start(t));
+            if (!mbar_wait(bar(B_KEMPTY0 + slot), (use & 1u) ^ 1u, st, 41)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(bar(B_KFULL0 + slot), 2 * kHalf);
+            for (int h = 0; h < 2; ++h)
+              tma_load_2d(&tmK, sbase + kKOff + (2 * slot + h) * kHalf, bar(B_KFULL0 + slot), h * 64, y);
+            if (!mbar_wait(bar(B_VEMPTY0 + slot), (use & 1u) ^ 1u, st, 42)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(bar(B_VFULL0 + slot), 2 * kHalf);
+            for (int h = 0; h < 2; ++h)
+              tma_load_2d(&tmV, sbase + kVOff + (2 * slot + h) * kHalf, bar(B_VFULL0 + slot), h * 64, y);
+          }
+        }
+        if (!ok) {
+          // leave no copy in flight into shared memory this CTA is giving up:
+          // wait (bounded) for the last phase armed on every full barrier
+#pragma unroll
+          for (int X = 0; X < 2; ++X)
+            if (n_xi[X] > 0) mbar_wait(bar(B_QFULL0 + X), (n_xi[X] - 1) & 1u, st, 50);
+          for (uint32_t k = n_kv > 2 ? n_kv - 2 : 0; k < n_kv; ++k) {
+            mbar_wait(bar(B_KFULL0 + (k & 1)), (k >> 1) & 1u, st, 50);
+            mbar_wait(bar(B_VFULL0 + (k & 1)), (k >> 1) & 1u, st, 50);
+          }
+        }
+      }
+    } else if (warp == kWarpMma) {
+      // ---- MMA issuer
+      if (lane == 0) {
+        struct Pending {  // P V of a sub-tile's tile, issued at the next tile
+          int valid, first, last, release_v;
+          uint32_t slot, use, xt;
+        };
+        Pending pend[2] = {};
+        uint32_t n_kv = 0, n_xt[2] = {0, 0}, n_xi[2] = {0, 0};
+        bool ok = true;
+        auto issue_pv = [&](int X) -> bool {
+          Pending& p = pend[X];
+          if (!mbar_wait(bar(B_PFULL0 + X), p.xt & 1u, st, 43)) return false;
+          if (!mbar_wait(bar(B_VFULL0 + p.slot), p.use & 1u, st, 44)) return false;
+          tc_fence_after();
+          const uint32_t tS = tmem + 128 * X, tO = tmem + 256 + 128 * X;
+#pragma unroll
+          for (int k = 0; k < kKeys / 16; ++k) {
+            const uint64_t db = smem_desc_sw128_mn(sbase + kVOff + 2 * p.slot * kHalf + k * 2048, kHalf);
+            tc_mma_f16_ts(tO, tS + 8 * k, db, kIdescPV, (p.first && k == 0) ? 0u : 1u);
+          }
+          if (p.last) tc_commit(bar(B_OFULL0 + X));
+          if (p.release_v) tc_commit(bar(B_VEMPTY0 + p.slot));
+          p.valid = 0;
+          return true;
+        };
+        for (ItemStream<G> is(plan, blockIdx.x, gridDim.x, b); is.valid() && ok;) {
+          const Item m = is.next();
+          const int nx = 1 + m.has_b;
+          for (int t = 0; t < m.n_tiles && ok; ++t, ++n_kv) {
+            const uint32_t slot = n_kv & 1, use = n_kv >> 1;
+#pragma unroll 1
+            for (int X = 0; X < 2; ++X) {
+              // P V of this sub-tile's previous tile first: S of this tile
+              // overwrites the P it reads
+              if (pend[X].valid && !issue_pv(X)) {
+                ok = false;
+                break;
+              }
+              if (X >= nx) continue;
+              if (t == 0 && !mbar_wait(bar(B_QFULL0 + X), n_xi[X] & 1u, st, 45)) {
+                ok = false;
+                break;
+              }
+              if (X == 0 && !mbar_wait(bar(B_KFULL0 + slot), use & 1u, st, 46)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+#pragma unroll
+              for (int k = 0; k < kHD / 16; ++k) {
+                const uint64_t da = smem_desc_sw128(sbase + kQOff + (2 * X + (k >> 2)) * kHalf + (k & 3) * 32);
+                const uint64_t db = smem_desc_sw128(sbase + kKOff + (2 * slot + (k >> 2)) * kHalf + (k & 3) * 32);
+                tc_mma_f16(tmem + 128 * X, da, db, kIdescS, k > 0 ? 1u : 0u);
+              }
+              tc_commit(bar(B_SFULL0 + X));
+              const bool last = t == m.n_tiles - 1;
+              if (last) {
+                tc_commit(bar(B_QEMPTY0 + X));  // Q_X free once these S are done
+                ++n_xi[X];
+              }
+              pend[X] = Pending{1, t == 0, last, X == nx - 1, slot, use, n_xt[X]};
+              ++n_xt[X];
+            }
+            if (ok) tc_commit(bar(B_KEMPTY0 + slot));  // both S of this tile issued
+          }
+        }
+#pragma unroll 1
+        for (int X = 0; X < 2; ++X)
+          if (ok && pend[X].valid && !issue_pv(X)) ok = false;
+        // no tensor-core operation of this CTA may outlive its TMEM
+        tc_commit(bar(B_DRAIN));
+        mbar_wait(bar(B_DRAIN), 0, st, 47);
+      }
     }
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kWarpMma) tmem_dealloc(tmem, kTmemCols);
 }
 
-int attention_tc_rows_per_item(int group) { return kSlots / group; }
+int attention_tc_rows_per_item(int group) { return 2 * kSub / group; }
 int attention_tc_smem_bytes() { return kSmem; }
 
 cudaError_t attention_tc_setup() {

@@ -92,7 +92,7 @@ cudaError_t debug_mask(const PlanHdr* plan, int request, uint8_t* out, int64_t t
 cudaError_t attention_f32(const PlanHdr* plan, const float* q, const float* kc, const float* vc, int64_t kv_rows,
                           int n_q_heads, int n_kv_heads, int hd, float scale, float* o, int max_rows,
                           cudaStream_t s);
-// tcgen05 attention (fp16 path): items of 128 query slots, KV tiles of 128 keys
+// tcgen05 attention (fp16 path): items of two 128-slot query sub-tiles, KV tiles of 128 keys
 cudaError_t attention_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const PlanHdr* plan,
                          int64_t kv_rows, int n_q_heads, int n_kv_heads, float scale, __half* o, DevStatus* st,
                          int grid, cudaStream_t s);

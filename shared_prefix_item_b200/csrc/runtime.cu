@@ -24,7 +24,7 @@ using namespace duolm;
 namespace {
 
 constexpr int kMaxPos = 32768;   // position ids must stay below this
-constexpr int kKvPad = 128;      // spare KV rows so a 128-key tile never leaves the buffer
+constexpr int kKvPad = 256;      // spare KV rows so the branch key tiles of an item never leave the buffer
 constexpr int kPerLayer = 11;
 
 struct LayerW {

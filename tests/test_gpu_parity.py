@@ -129,11 +129,14 @@ def test_q2_layout_mask_gather_bit_exact():
     (311, 1, 0, 1, 1, 1, 1),            # L = 1, K = 1
     (312, 3, (1, 6), (3, 20), (5, 40), 1, 7),
     (313, 2, (0, 4), (1, 30), (1, 20), 4, 3),
-    (314, 2, 2, 28, 33, 1, 1),          # L = 63: prefix one short of a key tile
-    (315, 1, 1, 60, 64, 1, 0),          # L = 64 exactly, branch rows span 2 items
+    (314, 2, 2, 28, 33, 1, 1),          # L = 63: prefix one short of a query sub-tile
+    (315, 1, 1, 60, 64, 1, 0),          # L = 64, K = 64: every item fills sub-tile A only
     (316, 2, 3, (40, 45), (30, 70), 2, 5),  # L > 128: several key tiles, ragged tail
-    (317, 1, 1, 60, 9, 32, 2),          # b = 32: half an attention item
-    (318, 1, 1, 70, 3, 64, 2),          # b = 64: the longest branch the kernel takes
+    (317, 1, 1, 60, 9, 32, 2),          # b = 32: a quarter of an attention item
+    (318, 1, 1, 70, 2, 128, 2),         # b = 128: the longest branch the kernel takes
+    (3101, 1, 1, 122, 200, 1, 2),       # L = 128 (one full item), branch rows span two items
+    (3105, 4, 1, (120, 125), (60, 70), 1, 2),  # L in {126, ..., 129}: item and key-tile edges
+    (3112, 1, 1, 60, 3, 96, 2),         # b = 96: one candidate per item, split across sub-tiles
 ])
 def test_q2_ragged_scores(seed, n_req, n_hist, fb, K, b, n_instr):
     wl = W.custom(Q2, Q2_ITEMS, seed, n_req, n_hist, fb, K, b, n_instr=n_instr, n_header=2)
@@ -184,7 +187,7 @@ def test_host_validation_errors():
         rk.score(p, np.array([1, 5, len(p)]), b, co, 1)
     assert e.value.code == -3
     with pytest.raises(S.DuolmError) as e:
-        rk.score(p, po, np.zeros(8 * 65, np.int32), co, 65)  # branch longer than an item
+        rk.score(p, po, np.zeros(8 * 129, np.int32), co, 129)  # branch longer than an item
     assert e.value.code == -1
     # the context is still usable
     ref = rk.score_workload(wl)
