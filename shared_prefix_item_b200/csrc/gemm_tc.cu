@@ -14,6 +14,8 @@
 // tile i+1.  Every mbarrier wait is bounded (see common.cuh).
 #include <cstdio>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -27,13 +29,16 @@ constexpr int kBK = 64;  // one 128-byte swizzle row of fp16
 // the pair MMAs (M = 256), each CTA's TMEM receives its 128 accumulator rows.
 // Tiles are visited N-fastest, so the pairs running at the same time share
 // an A row block and it is read from DRAM once.
-template <int BN>
+// An epilogue may ask for shared-memory scratch per epilogue warp (then the
+// ring is shallower, so the CTA stays near 197 KB of shared memory).
+template <int BN, class Epi>
 struct TcCfg {
-  static constexpr int STAGES = 6;
+  static constexpr int STAGES = Epi::STAGES;
   static constexpr int A_BYTES = kBM * kBK * 2;        // this CTA's 128 rows of A
   static constexpr int B_BYTES = (BN / 2) * kBK * 2;   // this CTA's half of the B tile
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  static constexpr int EPI_OFF = STAGES * STAGE_BYTES;
+  static constexpr int BAR_OFF = EPI_OFF + 4 * Epi::EG * Epi::SCRATCH_PER_WARP;
   static constexpr int SMEM = BAR_OFF + 256 + 1024;    // barriers + alignment slack
   static constexpr uint32_t TMEM_COLS = 2 * BN;        // two accumulator buffers
   static constexpr uint32_t IDESC = idesc_f16_f32(2 * kBM, BN);
@@ -43,7 +48,8 @@ struct TcCfg {
 // fused epilogues.  EG groups of four warps share each tile: group g handles
 // columns [g * BN / EG, (g + 1) * BN / EG) (for QKV, head g of the tile).
 // `taddr` addresses this thread's row, column 0 of the tile's accumulator;
-// all lanes of a warp execute the TMEM loads.
+// all lanes of a warp execute the TMEM loads.  `scratch` is this warp's
+// shared-memory scratch (SCRATCH_PER_WARP bytes).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float silu_fast(float g) {
   return __fdividef(g, 1.0f + fast_exp2(-1.4426950408889634f * g));
@@ -63,73 +69,103 @@ __device__ __forceinline__ float row_rnorm(const float* ssp, int n_slots, int ro
   return 1.0f / sqrtf(ss * inv_d + eps);
 }
 
+// x += scale * acc (the residual stream, fp32) and, for the next norm,
+// xg = fp16(x * g_next) with per-64-column partial sums of x^2.  The
+// accumulator arrives one row per thread; each warp turns its 32 x 32 block
+// around in shared memory so that the residual is read and written a row
+// segment of 128 bytes per 8 threads (four full lines per warp access)
+// instead of 32 rows per access.
 struct EpiResid {
   EpiResidArgs a;
-  static constexpr int EG = 4;
+  static constexpr int EG = 2;
+  static constexpr int STAGES = 5;
+  static constexpr int kPad = 36;  // words per scratch row: 16-byte stores and loads without bank conflicts
+  static constexpr int SCRATCH_PER_WARP = 32 * kPad * 4;
   template <int BN>
-  __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, int g, bool row_ok, const PlanHdr*,
-                                      DevStatus* st) const {
+  __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, int g, bool, const PlanHdr*, DevStatus* st,
+                                      uint8_t* scratch, int M) const {
     constexpr int W = BN / EG;
-    float ss = 0.f;
+    static_assert(W % 64 == 0, "a group covers whole 64-column norm slots");
+    const int lane = threadIdx.x & 31;
+    const int row0 = row - lane;      // the warp's first row
+    const int cq = (lane & 7) * 4;    // this thread's 4 columns of a 32-column chunk
+    const int rsub = lane >> 3;       // and its rows row0 + 4 i + rsub, i = 0..7
+    float* buf = reinterpret_cast<float*>(scratch);
+    float ss[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ss[i] = 0.f;
 #pragma unroll 1
     for (int c = g * W; c < (g + 1) * W; c += 32) {
-      // the residual loads do not depend on the accumulator: issue them first
-      float4* p = reinterpret_cast<float4*>(a.x + (int64_t)(row_ok ? row : 0) * a.ldx + n0 + c);
-      float4 t[8];
-      if (row_ok) {
+      // residual block: rows row0 + 4 i + rsub, columns c + cq .. + 3 (the
+      // loads do not depend on the accumulator: issue them first)
+      float4 xr[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) t[j] = p[j];
+      for (int i = 0; i < 8; ++i) {
+        const int rr = row0 + 4 * i + rsub;
+        xr[i] = rr < M ? *reinterpret_cast<const float4*>(a.x + (int64_t)rr * a.ldx + n0 + c + cq)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
       }
       uint32_t vr[32];
       tmem_ld32_async(taddr + c, vr);
       tmem_wait_ld();
-      float v[32];
+      __syncwarp();  // the previous chunk's reads of the scratch are done
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        tmem_ld_fence(vr[j]);
-        v[j] = __uint_as_float(vr[j]);
+      for (int q = 0; q < 8; ++q) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tmem_ld_fence(vr[4 * q + j]);
+        *reinterpret_cast<float4*>(buf + lane * kPad + 4 * q) =
+            make_float4(__uint_as_float(vr[4 * q]), __uint_as_float(vr[4 * q + 1]), __uint_as_float(vr[4 * q + 2]),
+                        __uint_as_float(vr[4 * q + 3]));
       }
-      if (row_ok) {
+      __syncwarp();
+      float4 gn = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (a.xg) gn = *reinterpret_cast<const float4*>(a.g_next + n0 + c + cq);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          t[j].x += v[4 * j + 0] * a.scale;
-          t[j].y += v[4 * j + 1] * a.scale;
-          t[j].z += v[4 * j + 2] * a.scale;
-          t[j].w += v[4 * j + 3] * a.scale;
-          p[j] = t[j];
-        }
-        if (a.xg) {
-          const float* gn = a.g_next + n0 + c;
-          uint32_t pk[16];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            ss += t[j].x * t[j].x;
-            ss += t[j].y * t[j].y;
-            ss += t[j].z * t[j].z;
-            ss += t[j].w * t[j].w;
-            const __half2 h0 = __halves2half2(to_half_checked(t[j].x * gn[4 * j + 0], st, 23),
-                                              to_half_checked(t[j].y * gn[4 * j + 1], st, 23));
-            const __half2 h1 = __halves2half2(to_half_checked(t[j].z * gn[4 * j + 2], st, 23),
-                                              to_half_checked(t[j].w * gn[4 * j + 3], st, 23));
-            pk[2 * j] = *reinterpret_cast<const uint32_t*>(&h0);
-            pk[2 * j + 1] = *reinterpret_cast<const uint32_t*>(&h1);
+      for (int i = 0; i < 8; ++i) {
+        const int rl = 4 * i + rsub;
+        const int rr = row0 + rl;
+        const float4 acc = *reinterpret_cast<const float4*>(buf + rl * kPad + cq);
+        float4 t = xr[i];
+        t.x += acc.x * a.scale;
+        t.y += acc.y * a.scale;
+        t.z += acc.z * a.scale;
+        t.w += acc.w * a.scale;
+        if (rr < M) {
+          *reinterpret_cast<float4*>(a.x + (int64_t)rr * a.ldx + n0 + c + cq) = t;
+          if (a.xg) {
+            ss[i] += t.x * t.x + t.y * t.y + t.z * t.z + t.w * t.w;
+            const __half2 h0 = __halves2half2(to_half_checked(t.x * gn.x, st, 23), to_half_checked(t.y * gn.y, st, 23));
+            const __half2 h1 = __halves2half2(to_half_checked(t.z * gn.z, st, 23), to_half_checked(t.w * gn.w, st, 23));
+            *reinterpret_cast<uint2*>(a.xg + (int64_t)rr * a.ldx + n0 + c + cq) =
+                make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
           }
-          uint4* q = reinterpret_cast<uint4*>(a.xg + (int64_t)row * a.ldx + n0 + c);
+        }
+      }
+      if (a.xg && (c & 63) == 32) {
+        // a 64-column slot is complete: sum each row over its 8 threads
 #pragma unroll
-          for (int j = 0; j < 4; ++j) q[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        for (int i = 0; i < 8; ++i) {
+          float v = ss[i];
+          v += __shfl_xor_sync(0xffffffffu, v, 1);
+          v += __shfl_xor_sync(0xffffffffu, v, 2);
+          v += __shfl_xor_sync(0xffffffffu, v, 4);
+          const int rr = row0 + 4 * i + rsub;
+          if ((lane & 7) == 0 && rr < M) a.ssp[(int64_t)rr * a.n_slots + (n0 + c) / 64] = v;
+          ss[i] = 0.f;
         }
       }
     }
-    if (row_ok && a.xg) a.ssp[(int64_t)row * a.n_slots + (n0 / BN) * EG + g] = ss;
   }
 };
 
 struct EpiSwiglu {
   EpiSwigluArgs a;
   static constexpr int EG = 4;
+  static constexpr int STAGES = 6;
+  static constexpr int SCRATCH_PER_WARP = 0;
   template <int BN>
   __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, int g, bool row_ok, const PlanHdr*,
-                                      DevStatus* st) const {
+                                      DevStatus* st, uint8_t*, int) const {
     constexpr int H = BN / 2;   // gate columns [0, H), up columns [H, BN)
     constexpr int W = H / EG;   // outputs of this group
     const int out0 = n0 / 2;
@@ -171,9 +207,11 @@ struct EpiSwiglu {
 struct EpiQkv {
   EpiQkvArgs a;
   static constexpr int EG = 2;  // one head of the 256-column tile per group
+  static constexpr int STAGES = 6;
+  static constexpr int SCRATCH_PER_WARP = 0;
   template <int BN>
   __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, int g, bool row_ok, const PlanHdr* plan,
-                                      DevStatus* st) const {
+                                      DevStatus* st, uint8_t*, int) const {
     const int gc = n0 + 128 * g;
     const uint32_t base = taddr + 128 * g;
     // weight scale times the input row's RMSNorm factor
@@ -271,7 +309,7 @@ template <int BN, class Epi>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 128 * Epi::EG, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int Kdim,
                    int N, const PlanHdr* __restrict__ plan, const Epi epi, DevStatus* st) {
-  using C = TcCfg<BN>;
+  using C = TcCfg<BN, Epi>;
   constexpr int EG = Epi::EG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -397,7 +435,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 128 * Epi::EG, 
         const int m_blk = tile / n_tiles, n_blk = tile % n_tiles;
         const int row = m_blk * 2 * kBM + (int)rank * kBM + q4 * 32 + lane;
         const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q4 * 32) << 16);
-        epi.template run<BN>(taddr, row, n_blk * BN, group, row < M, plan, st);
+        epi.template run<BN>(taddr, row, n_blk * BN, group, row < M, plan, st,
+                             smem + C::EPI_OFF + (warp - 2) * Epi::SCRATCH_PER_WARP, M);
         // the accumulator may be overwritten once every epilogue thread of
         // the pair has read it; the reads are ordered by the tcgen05 fence,
         // the global stores need no ordering with the MMA
@@ -477,33 +516,35 @@ bool make_tmap_f16_3d(CUtensorMap* map, const void* base, const uint64_t dims[3]
   return true;
 }
 
-int gemm_tc_smem_bytes(int bn) { return bn == 256 ? TcCfg<256>::SMEM : TcCfg<128>::SMEM; }
+int gemm_tc_smem_bytes(int) {
+  return std::max(TcCfg<256, EpiResid>::SMEM, std::max(TcCfg<256, EpiSwiglu>::SMEM, TcCfg<256, EpiQkv>::SMEM));
+}
 
 cudaError_t gemm_tc_setup() {
   cudaError_t e;
   if ((e = cudaFuncSetAttribute(gemm_tc_kernel<256, EpiResid>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                TcCfg<256>::SMEM)) != cudaSuccess)
+                                TcCfg<256, EpiResid>::SMEM)) != cudaSuccess)
     return e;
   if ((e = cudaFuncSetAttribute(gemm_tc_kernel<256, EpiSwiglu>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                TcCfg<256>::SMEM)) != cudaSuccess)
+                                TcCfg<256, EpiSwiglu>::SMEM)) != cudaSuccess)
     return e;
   return cudaFuncSetAttribute(gemm_tc_kernel<256, EpiQkv>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              TcCfg<256>::SMEM);
+                              TcCfg<256, EpiQkv>::SMEM);
 }
 
 cudaError_t gemm_tc_resid(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
                           EpiResidArgs e, DevStatus* st, int grid, cudaStream_t s) {
-  gemm_tc_kernel<256, EpiResid><<<grid, 64 + 128 * EpiResid::EG, TcCfg<256>::SMEM, s>>>(a, b, K, N, plan, EpiResid{e}, st);
+  gemm_tc_kernel<256, EpiResid><<<grid, 64 + 128 * EpiResid::EG, TcCfg<256, EpiResid>::SMEM, s>>>(a, b, K, N, plan, EpiResid{e}, st);
   return cudaGetLastError();
 }
 cudaError_t gemm_tc_swiglu(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
                            EpiSwigluArgs e, DevStatus* st, int grid, cudaStream_t s) {
-  gemm_tc_kernel<256, EpiSwiglu><<<grid, 64 + 128 * EpiSwiglu::EG, TcCfg<256>::SMEM, s>>>(a, b, K, N, plan, EpiSwiglu{e}, st);
+  gemm_tc_kernel<256, EpiSwiglu><<<grid, 64 + 128 * EpiSwiglu::EG, TcCfg<256, EpiSwiglu>::SMEM, s>>>(a, b, K, N, plan, EpiSwiglu{e}, st);
   return cudaGetLastError();
 }
 cudaError_t gemm_tc_qkv(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
                         EpiQkvArgs e, DevStatus* st, int grid, cudaStream_t s) {
-  gemm_tc_kernel<256, EpiQkv><<<grid, 64 + 128 * EpiQkv::EG, TcCfg<256>::SMEM, s>>>(a, b, K, N, plan, EpiQkv{e}, st);
+  gemm_tc_kernel<256, EpiQkv><<<grid, 64 + 128 * EpiQkv::EG, TcCfg<256, EpiQkv>::SMEM, s>>>(a, b, K, N, plan, EpiQkv{e}, st);
   return cudaGetLastError();
 }
 
