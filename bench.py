@@ -109,6 +109,48 @@ def attention_flops(shape: W.ModelShape, wl: W.Workload, independent: bool) -> f
     return 4.0 * shape.head_dim * shape.n_q_heads * attention_pairs(wl, independent) * shape.n_layers
 
 
+def class_flops(shape: W.ModelShape, wl: W.Workload, T: int, independent: bool) -> dict:
+    """Algorithmic FLOPs per step of each kernel class (multiply-add = 2)."""
+    d, qd, kd, F, L = shape.d, shape.q_dim, shape.kv_dim, shape.ffn, shape.n_layers
+    return {
+        "gemm_qkv": 2.0 * T * d * (qd + 2 * kd) * L,
+        "gemm_o": 2.0 * T * qd * d * L,
+        "gemm_gate_up": 2.0 * T * d * 2 * F * L,
+        "gemm_down": 2.0 * T * F * d * L,
+        "attention": attention_flops(shape, wl, independent),
+    }
+
+
+KERNEL_SOURCES = {  # the files a kernel class is built from (its ncu traffic is stale once they change)
+    "gemm_qkv": ("gemm_tc.cu", "common.cuh"), "gemm_o": ("gemm_tc.cu", "common.cuh"),
+    "gemm_gate_up": ("gemm_tc.cu", "common.cuh"), "gemm_down": ("gemm_tc.cu", "common.cuh"),
+    "attention": ("attention_tc.cu", "common.cuh"),
+}
+
+
+def source_hash(kind: str) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kind]:
+        with open(os.path.join(ROOT, "shared_prefix_item_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def captured_traffic(kind: str, config: str):
+    """DRAM bytes per launch (read + write) of a kernel class from the committed
+    ncu summary, or None when there is none for this workload or the kernel's
+    sources changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        t = json.load(f).get(config, {}).get(kind)
+    if not t or t.get("source_hash") != source_hash(kind):
+        return None
+    return t["dram_bytes_per_launch"]
+
+
 def attention_bytes(shape: W.ModelShape, T: int) -> float:
     # q read, k and v read once, o written (fp16), per layer
     return 2.0 * T * (2 * shape.q_dim + 2 * shape.kv_dim) * shape.n_layers
@@ -334,29 +376,36 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     steps_prof = max(2, min(args.steps, 5))
     pk = peaks()
     indep = mode == S.MODE_INDEPENDENT
-    g_ms = sum(prof[k][0] for k in ("gemm_qkv", "gemm_o", "gemm_gate_up", "gemm_down")) / steps_prof
-    g_n = sum(prof[k][1] for k in ("gemm_qkv", "gemm_o", "gemm_gate_up", "gemm_down")) / steps_prof
-    a_ms = prof["attention"][0] / steps_prof
-    a_n = prof["attention"][1] / steps_prof
-    gf = gemm_flops(shape, T)
-    af = attention_flops(shape, wl, indep)
+    cf = class_flops(shape, wl, T, indep)
+    gf = sum(v for k, v in cf.items() if k != "attention")
+    af = cf["attention"]
     kernels = {k: {"ms_per_step": round(v[0] / steps_prof, 4), "launches_per_step": v[1] // steps_prof}
                for k, v in prof.items()}
     tot_ms = sum(v["ms_per_step"] for v in kernels.values())
     for v in kernels.values():
         v["share"] = round(v["ms_per_step"] / tot_ms, 4) if tot_ms else None
-    gemm_roof = {"bound": "tensor", "achieved": gf / (g_ms / 1e3) / 1e12, "peak": pk["tc_sustained"],
-                 "unit": "TFLOP/s", "kernel": "gemm_tc_kernel (QKV, O, gate/up, down)",
-                 "launches_per_step": g_n, "flops_per_launch": gf / max(g_n, 1)}
-    attn_roof = {"bound": "tensor", "achieved": af / (a_ms / 1e3) / 1e12, "peak": pk["tc_sustained"],
-                 "unit": "TFLOP/s", "kernel": "attention_f16_kernel",
-                 "launches_per_step": a_n, "flops_per_launch": af / max(a_n, 1),
-                 "hbm_gbs_algorithmic": attention_bytes(shape, T) / (a_ms / 1e3) / 1e9}
-    for r in (gemm_roof, attn_roof):
+    names = {"gemm_qkv": "gemm_tc_kernel<EpiQkv> (QKV projection, QK-norm, RoPE)",
+             "gemm_o": "gemm_tc_kernel<EpiResid> (O projection + residual)",
+             "gemm_gate_up": "gemm_tc_kernel<EpiSwiglu> (gate/up projection + SwiGLU)",
+             "gemm_down": "gemm_tc_kernel<EpiResid> (down projection + residual)",
+             "attention": "attention_tc_kernel (shared-prefix tree attention)"}
+    roofs = {}
+    for k, fl in cf.items():
+        ms_k = prof[k][0] / steps_prof
+        n_k = max(prof[k][1] // steps_prof, 1)
+        if ms_k <= 0:
+            continue
+        r = {"bound": "tensor", "achieved": fl / (ms_k / 1e3) / 1e12, "peak": pk["tc_sustained"],
+             "unit": "TFLOP/s", "kernel": names[k], "launches_per_step": n_k, "flops_per_launch": fl / n_k,
+             "us_per_launch": ms_k * 1e3 / n_k,
+             "peak_note": f"{pk['src']} sustained bf16 dense (fp16 runs at the bf16 rate)",
+             "traffic": captured_traffic(k, args.config)}
         r["frac"] = r["achieved"] / r["peak"]
-        r["peak_note"] = f"{pk['src']} sustained bf16 dense (fp16 runs at the bf16 rate)"
-        r["traffic"] = None
-    dominant = gemm_roof if g_ms >= a_ms else attn_roof
+        if k == "attention":
+            r["hbm_gbs_algorithmic"] = attention_bytes(shape, T) / (ms_k / 1e3) / 1e9
+        roofs[k] = r
+    dom_key = max(roofs, key=lambda k: prof[k][0])
+    dominant = roofs[dom_key]
     step_roof_ms = max((gf + af) / (pk["tc_sustained"] * 1e12), 0.0) * 1e3
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu:
@@ -376,7 +425,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
             "roofline_step": {"flops_per_step": gf + af, "ms_at_peak": step_roof_ms,
                               "frac": step_roof_ms / ms_max, "peak": pk["tc_sustained"],
                               "unit": "TFLOP/s", "note": "whole step vs max(FLOPs/peak, bytes/HBM BW)"},
-            "roofline_other": attn_roof if dominant is gemm_roof else gemm_roof,
+            "roofline_other": {k: v for k, v in roofs.items() if k != dom_key},
             "kernels": kernels,
             "gpu_launches": launches * args.steps,
             "clocks": clk.summary(),

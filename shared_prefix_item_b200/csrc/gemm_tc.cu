@@ -49,7 +49,9 @@ struct TcCfg {
 // columns [g * BN / EG, (g + 1) * BN / EG) (for QKV, head g of the tile).
 // `taddr` addresses this thread's row, column 0 of the tile's accumulator;
 // all lanes of a warp execute the TMEM loads.  `scratch` is this warp's
-// shared-memory scratch (SCRATCH_PER_WARP bytes).
+// shared-memory scratch (SCRATCH_PER_WARP bytes).  prefetch() runs before the
+// wait for the accumulator and loads what does not depend on it (the input
+// row's norm factor, positions, tables); its result is passed to run().
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float silu_fast(float g) {
   return __fdividef(g, 1.0f + fast_exp2(-1.4426950408889634f * g));
@@ -75,15 +77,44 @@ __device__ __forceinline__ float row_rnorm(const float* ssp, int n_slots, int ro
 // around in shared memory so that the residual is read and written a row
 // segment of 128 bytes per 8 threads (four full lines per warp access)
 // instead of 32 rows per access.
+// Warp store of 32 rows x 128 bytes: thread `lane` holds row `lane` as 32
+// words; the rows go out through a padded shared-memory scratch (36 words a
+// row: 16-byte accesses without bank conflicts) so that eight threads store
+// one row's 128 bytes, four full lines per warp access.  dst(r) is the
+// 16-byte-aligned destination of row r of the warp, or null to skip it.
+constexpr int kScratchPad = 36;
+constexpr int kScratchPerWarp = 32 * kScratchPad * 4;
+template <class Dst>
+__device__ __forceinline__ void warp_store_rows_128B(uint32_t* buf, const uint32_t (&v)[32], Dst dst) {
+  const int lane = threadIdx.x & 31;
+  __syncwarp();  // earlier reads of the scratch are done
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    *reinterpret_cast<uint4*>(buf + lane * kScratchPad + 4 * q) = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = 4 * i + (lane >> 3);
+    const uint4 w = *reinterpret_cast<const uint4*>(buf + r * kScratchPad + (lane & 7) * 4);
+    uint4* p = dst(r);
+    if (p) p[lane & 7] = w;
+  }
+}
+
 struct EpiResid {
   EpiResidArgs a;
   static constexpr int EG = 2;
   static constexpr int STAGES = 5;
-  static constexpr int kPad = 36;  // words per scratch row: 16-byte stores and loads without bank conflicts
-  static constexpr int SCRATCH_PER_WARP = 32 * kPad * 4;
+  static constexpr int kPad = kScratchPad;
+  static constexpr int SCRATCH_PER_WARP = kScratchPerWarp;
+  struct Pre {};
+  template <int BN>
+  __device__ __forceinline__ Pre prefetch(int, int, int, bool, const PlanHdr*, DevStatus*) const {
+    return Pre{};
+  }
   template <int BN>
   __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, int g, bool, const PlanHdr*, DevStatus* st,
-                                      uint8_t* scratch, int M) const {
+                                      uint8_t* scratch, int M, const Pre&) const {
     constexpr int W = BN / EG;
     static_assert(W % 64 == 0, "a group covers whole 64-column norm slots");
     const int lane = threadIdx.x & 31;
@@ -160,44 +191,50 @@ struct EpiResid {
 
 struct EpiSwiglu {
   EpiSwigluArgs a;
-  static constexpr int EG = 4;
-  static constexpr int STAGES = 6;
-  static constexpr int SCRATCH_PER_WARP = 0;
+  static constexpr int EG = 2;
+  static constexpr int STAGES = 5;
+  static constexpr int SCRATCH_PER_WARP = kScratchPerWarp;
+  struct Pre {
+    float sc;  // weight scale times the input row's RMSNorm factor
+  };
+  template <int BN>
+  __device__ __forceinline__ Pre prefetch(int row, int, int, bool row_ok, const PlanHdr*, DevStatus*) const {
+    return Pre{row_ok ? a.scale * row_rnorm(a.ssp, a.n_slots, row, a.inv_d, a.eps) : 0.f};
+  }
   template <int BN>
   __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, int g, bool row_ok, const PlanHdr*,
-                                      DevStatus* st, uint8_t*, int) const {
+                                      DevStatus* st, uint8_t* scratch, int M, const Pre& pre) const {
     constexpr int H = BN / 2;   // gate columns [0, H), up columns [H, BN)
-    constexpr int W = H / EG;   // outputs of this group
-    const int out0 = n0 / 2;
-    const float sc = row_ok ? a.scale * row_rnorm(a.ssp, a.n_slots, row, a.inv_d, a.eps) : 0.f;
-#pragma unroll 1
-    for (int c = g * W; c < (g + 1) * W; c += 32) {
+    constexpr int W = H / EG;   // outputs of this group: one 128-byte fp16 row segment
+    static_assert(W == 64, "one warp store per group");
+    const int out0 = n0 / 2 + g * W;
+    const float sc = pre.sc;
+    uint32_t packed[32];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int c = g * W + 32 * half;
       uint32_t gr[32], ur[32];
       tmem_ld32_async(taddr + c, gr);
       tmem_ld32_async(taddr + H + c, ur);
       tmem_wait_ld();
-      float gv[32], uv[32];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        tmem_ld_fence(gr[j]);
-        tmem_ld_fence(ur[j]);
-        gv[j] = __uint_as_float(gr[j]);
-        uv[j] = __uint_as_float(ur[j]);
-      }
-      if (row_ok) {
-        uint32_t packed[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float h0 = silu_fast(gv[2 * j] * sc) * (uv[2 * j] * sc);
-          const float h1 = silu_fast(gv[2 * j + 1] * sc) * (uv[2 * j + 1] * sc);
-          __half2 hh = __halves2half2(to_half_checked(h0, st, 20), to_half_checked(h1, st, 20));
-          packed[j] = *reinterpret_cast<uint32_t*>(&hh);
-        }
-        uint4* p = reinterpret_cast<uint4*>(a.h + (int64_t)row * a.ldh + out0 + c);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) p[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+      for (int j = 0; j < 16; ++j) {
+        tmem_ld_fence(gr[2 * j]);
+        tmem_ld_fence(gr[2 * j + 1]);
+        tmem_ld_fence(ur[2 * j]);
+        tmem_ld_fence(ur[2 * j + 1]);
+        const float h0 = silu_fast(__uint_as_float(gr[2 * j]) * sc) * (__uint_as_float(ur[2 * j]) * sc);
+        const float h1 = silu_fast(__uint_as_float(gr[2 * j + 1]) * sc) * (__uint_as_float(ur[2 * j + 1]) * sc);
+        __half2 hh = row_ok ? __halves2half2(to_half_checked(h0, st, 20), to_half_checked(h1, st, 20))
+                            : __halves2half2(__float2half_rn(0.f), __float2half_rn(0.f));
+        packed[16 * half + j] = *reinterpret_cast<uint32_t*>(&hh);
       }
     }
+    const int row0 = row - (int)(threadIdx.x & 31);
+    warp_store_rows_128B(reinterpret_cast<uint32_t*>(scratch), packed, [&](int r) -> uint4* {
+      const int rr = row0 + r;
+      return rr < M ? reinterpret_cast<uint4*>(a.h + (int64_t)rr * a.ldh + out0) : nullptr;
+    });
   }
 };
 
@@ -209,9 +246,14 @@ struct EpiQkv {
   static constexpr int EG = 2;  // one head of the 256-column tile per group
   static constexpr int STAGES = 6;
   static constexpr int SCRATCH_PER_WARP = 0;
+  struct Pre {};
+  template <int BN>
+  __device__ __forceinline__ Pre prefetch(int, int, int, bool, const PlanHdr*, DevStatus*) const {
+    return Pre{};
+  }
   template <int BN>
   __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, int g, bool row_ok, const PlanHdr* plan,
-                                      DevStatus* st, uint8_t*, int) const {
+                                      DevStatus* st, uint8_t*, int, const Pre&) const {
     const int gc = n0 + 128 * g;
     const uint32_t base = taddr + 128 * g;
     // weight scale times the input row's RMSNorm factor
@@ -430,13 +472,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 128 * Epi::EG, 
       for (int tile = pair; tile < num_tiles; tile += n_pairs, ++local) {
         const int acc = local & 1;
         const uint32_t use = (uint32_t)(local >> 1);
-        if (!mbar_wait_warp(tfull0 + 8 * acc, use & 1u, st, 4)) break;
-        tc_fence_after();
         const int m_blk = tile / n_tiles, n_blk = tile % n_tiles;
         const int row = m_blk * 2 * kBM + (int)rank * kBM + q4 * 32 + lane;
+        const typename Epi::Pre pre = epi.template prefetch<BN>(row, n_blk * BN, group, row < M, plan, st);
+        if (!mbar_wait_warp(tfull0 + 8 * acc, use & 1u, st, 4)) break;
+        tc_fence_after();
         const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q4 * 32) << 16);
         epi.template run<BN>(taddr, row, n_blk * BN, group, row < M, plan, st,
-                             smem + C::EPI_OFF + (warp - 2) * Epi::SCRATCH_PER_WARP, M);
+                             smem + C::EPI_OFF + (warp - 2) * Epi::SCRATCH_PER_WARP, M, pre);
         // the accumulator may be overwritten once every epilogue thread of
         // the pair has read it; the reads are ordered by the tcgen05 fence,
         // the global stores need no ordering with the MMA
