@@ -339,24 +339,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kWarpMma) {
       // ---- MMA issuer
       if (lane == 0) {
+        // (all state in named registers: runtime-indexed arrays would sit in
+        // local memory, and this thread's instruction path bounds the step)
         struct Pending {  // P V of a sub-tile's tile, issued at the next tile
           int valid, first, last, release_v;
           uint32_t slot, use, xt;
         };
-        Pending pend[2] = {};
-        uint32_t n_kv = 0, n_xt[2] = {0, 0}, n_xi[2] = {0, 0};
+        Pending pa{}, pb{};
+        uint32_t n_kv = 0, xt_a = 0, xt_b = 0, xi_a = 0, xi_b = 0;
         bool ok = true;
-        auto issue_pv = [&](int X) -> bool {
-          Pending& p = pend[X];
+        auto issue_pv = [&](int X, Pending& p) -> bool {
           if (!mbar_wait(bar(B_PFULL0 + X), p.xt & 1u, st, 43)) return false;
           if (!mbar_wait(bar(B_VFULL0 + p.slot), p.use & 1u, st, 44)) return false;
           tc_fence_after();
           const uint32_t tS = tmem + 128 * X, tO = tmem + 256 + 128 * X;
+          const uint32_t vbase = sbase + kVOff + 2 * p.slot * kHalf;
 #pragma unroll
-          for (int k = 0; k < kKeys / 16; ++k) {
-            const uint64_t db = smem_desc_sw128_mn(sbase + kVOff + 2 * p.slot * kHalf + k * 2048, kHalf);
-            tc_mma_f16_ts(tO, tS + 8 * k, db, kIdescPV, (p.first && k == 0) ? 0u : 1u);
-          }
+          for (int k = 0; k < kKeys / 16; ++k)
+            tc_mma_f16_ts(tO, tS + 8 * k, smem_desc_sw128_mn(vbase + k * 2048, kHalf), kIdescPV,
+                          (p.first && k == 0) ? 0u : 1u);
           if (p.last) tc_commit(bar(B_OFULL0 + X));
           if (p.release_v) tc_commit(bar(B_VEMPTY0 + p.slot));
           p.valid = 0;
@@ -367,16 +368,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int nx = 1 + m.has_b;
           for (int t = 0; t < m.n_tiles && ok; ++t, ++n_kv) {
             const uint32_t slot = n_kv & 1, use = n_kv >> 1;
-#pragma unroll 1
+            const bool last = t == m.n_tiles - 1;
+            const uint32_t kbase = sbase + kKOff + 2 * slot * kHalf;
+#pragma unroll
             for (int X = 0; X < 2; ++X) {
+              Pending& p = X == 0 ? pa : pb;
               // P V of this sub-tile's previous tile first: S of this tile
               // overwrites the P it reads
-              if (pend[X].valid && !issue_pv(X)) {
+              if (p.valid && !issue_pv(X, p)) {
                 ok = false;
                 break;
               }
               if (X >= nx) continue;
-              if (t == 0 && !mbar_wait(bar(B_QFULL0 + X), n_xi[X] & 1u, st, 45)) {
+              uint32_t& xi = X == 0 ? xi_a : xi_b;
+              uint32_t& xt = X == 0 ? xt_a : xt_b;
+              if (t == 0 && !mbar_wait(bar(B_QFULL0 + X), xi & 1u, st, 45)) {
                 ok = false;
                 break;
               }
@@ -385,27 +391,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
               }
               tc_fence_after();
+              const uint32_t qbase = sbase + kQOff + 2 * X * kHalf;
 #pragma unroll
-              for (int k = 0; k < kHD / 16; ++k) {
-                const uint64_t da = smem_desc_sw128(sbase + kQOff + (2 * X + (k >> 2)) * kHalf + (k & 3) * 32);
-                const uint64_t db = smem_desc_sw128(sbase + kKOff + (2 * slot + (k >> 2)) * kHalf + (k & 3) * 32);
-                tc_mma_f16(tmem + 128 * X, da, db, kIdescS, k > 0 ? 1u : 0u);
-              }
+              for (int k = 0; k < kHD / 16; ++k)
+                tc_mma_f16(tmem + 128 * X, smem_desc_sw128(qbase + (k >> 2) * kHalf + (k & 3) * 32),
+                           smem_desc_sw128(kbase + (k >> 2) * kHalf + (k & 3) * 32), kIdescS, k > 0 ? 1u : 0u);
               tc_commit(bar(B_SFULL0 + X));
-              const bool last = t == m.n_tiles - 1;
               if (last) {
                 tc_commit(bar(B_QEMPTY0 + X));  // Q_X free once these S are done
-                ++n_xi[X];
+                ++xi;
               }
-              pend[X] = Pending{1, t == 0, last, X == nx - 1, slot, use, n_xt[X]};
-              ++n_xt[X];
+              p = Pending{1, t == 0, last, X == nx - 1, slot, use, xt};
+              ++xt;
             }
             if (ok) tc_commit(bar(B_KEMPTY0 + slot));  // both S of this tile issued
           }
         }
-#pragma unroll 1
-        for (int X = 0; X < 2; ++X)
-          if (ok && pend[X].valid && !issue_pv(X)) ok = false;
+        if (ok && pa.valid && !issue_pv(0, pa)) ok = false;
+        if (ok && pb.valid && !issue_pv(1, pb)) ok = false;
         // no tensor-core operation of this CTA may outlive its TMEM
         tc_commit(bar(B_DRAIN));
         mbar_wait(bar(B_DRAIN), 0, st, 47);

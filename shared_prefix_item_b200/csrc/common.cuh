@@ -124,16 +124,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking test of the same condition (for issuers that poll several
+// barriers in turn).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // Wait for the phase of the given parity to complete; false (and the error
 // flag raised) after kWaitLimitNs.
+// Reading %globaltimer is slow (of the order of the handoffs being waited
+// for), so the clock is first read only after kSpinsBeforeClock unsuccessful
+// polls and then once per as many more.
+constexpr uint32_t kSpinsBeforeClock = 1024;
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, DevStatus* st, uint32_t where) {
-  if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0 = global_ns();
+  uint64_t t0 = 0;
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) {
-      raise_error(st, ERR_WAIT_TIMEOUT, where);
-      return false;
+    if ((i & (kSpinsBeforeClock - 1)) == 0) {
+      const uint64_t now = global_ns();
+      if (i == kSpinsBeforeClock) {
+        t0 = now;
+      } else if (now - t0 > kWaitLimitNs) {
+        raise_error(st, ERR_WAIT_TIMEOUT, where);
+        return false;
+      }
     }
   }
 }
