@@ -312,6 +312,17 @@ struct EpiQkv {
       tmem_ld16(base + c, x1);
       tmem_ld16(base + 64 + c, x2);
       if (row_ok) {
+        // this chunk's 16 + 16 norm gains as four 16-byte loads each (the
+        // same addresses in every lane: broadcasts)
+        float g1[16], g2[16];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 u = reinterpret_cast<const float4*>(gain + c)[q];
+          const float4 w = reinterpret_cast<const float4*>(gain + 64 + c)[q];
+          g1[4 * q] = u.x, g1[4 * q + 1] = u.y, g1[4 * q + 2] = u.z, g1[4 * q + 3] = u.w;
+          g2[4 * q] = w.x, g2[4 * q + 1] = w.y, g2[4 * q + 2] = w.z, g2[4 * q + 3] = w.w;
+        }
+        const float scr = sc * r;
         uint32_t o1[8], o2[8];
 #pragma unroll
         for (int j = 0; j < 16; j += 2) {
@@ -319,8 +330,8 @@ struct EpiQkv {
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int i = c + j + e;
-            const float a1 = (x1[j + e] * sc * r) * gain[i];
-            const float a2 = (x2[j + e] * sc * r) * gain[64 + i];
+            const float a1 = (x1[j + e] * scr) * g1[j + e];
+            const float a2 = (x2[j + e] * scr) * g2[j + e];
             const float2 t = cs[(int64_t)i * a.max_pos];
             r1[e] = a1 * t.x - a2 * t.y;
             r2[e] = a2 * t.x + a1 * t.y;
