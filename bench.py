@@ -227,10 +227,12 @@ class ClockSampler:
 # CPU oracle timing
 # ---------------------------------------------------------------------------
 
-def oracle_time(wl: W.Workload, requests, warmup: int = 1) -> tuple:
+def oracle_time(wl: W.Workload, requests, warmup: int = 1, independent_cands: int = 0) -> tuple:
     """Score the given requests with the oracle; returns (seconds per request,
     candidates).  `warmup` short calls first load the library and page in the
-    weights."""
+    weights.  With independent_cands > 0, only that many candidates of each
+    request are scored, in independent mode (each candidate's whole prefix +
+    branch sequence on its own)."""
     from oracle import ranker as R
     om = R.OracleModel(wl.model, W.model_weights(wl.model))
     rho = R.embedding_rho(om.embed)
@@ -250,13 +252,16 @@ def oracle_time(wl: W.Workload, requests, warmup: int = 1) -> tuple:
                          for i in ids.reshape(-1)], np.int32).reshape(ids.shape)
 
     local = [W.Request(rm(wl.requests[q].prefix_ids), rm(wl.requests[q].branch_ids)) for q in requests]
+    if independent_cands:
+        local = [W.Request(r.prefix_ids, r.branch_ids[:independent_cands]) for r in local]
+    score = R.score_independent if independent_cands else R.score_mis
     for _ in range(max(1, warmup)):
         R.score_mis(om, sub, W.Request(local[0].prefix_ids[:4], local[0].branch_ids[:1]))
     per = []
     n = 0
     for req in local:
         t = time.perf_counter()
-        R.score_mis(om, sub, req)
+        score(om, sub, req)
         per.append(time.perf_counter() - t)
         n += req.K
     return per, n
@@ -293,6 +298,77 @@ def run_reference(args, rank: int, world: int) -> None:
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+GATHER_LOOKUPS = 4_194_304
+GATHER_TABLE_ROWS = 1_000_000
+
+
+def run_gather(args, rank: int, world: int, local_rank: int) -> None:
+    """The VID gather alone (duolm_gather): GATHER_LOOKUPS Zipf(1.1) lookups
+    over a GATHER_TABLE_ROWS-row FP16 item table, each writing the fp32 row,
+    its fp16 normed operand and its sum of squares; HBM bound."""
+    import torch
+
+    import shared_prefix_item_b200 as S
+    torch.cuda.set_device(local_rank)
+    shape = W.QWEN3_06B
+    stream = torch.cuda.Stream()
+    torch.cuda.set_stream(stream)
+    rk = S.Ranker(shape, W.model_weights(shape), device=local_rank, stream=stream.cuda_stream)
+    # a 1M-row table: 10k rows through the library's own interface, tiled
+    # (the values do not matter to the measurement, the size and the access
+    # pattern do)
+    base_rows = 10_000
+    rk.vid_table_build(W.item_vectors(base_rows, shape.d), 0.0, rk.embedding_rho())
+    rows = np.tile(rk.debug_table(base_rows), (GATHER_TABLE_ROWS // base_rows, 1))
+    rk.vid_table_load(rows)
+    del rows
+    n, d = GATHER_LOOKUPS, shape.d
+    ids = torch.from_numpy((shape.vocab + W.zipf_lookups(n, GATHER_TABLE_ROWS)).astype(np.int32)).cuda()
+    x = torch.empty((n, d), dtype=torch.float32, device="cuda")
+    xg = torch.empty((n, d), dtype=torch.int16, device="cuda")
+    ssp = torch.empty((n, d // 64), dtype=torch.float32, device="cuda")
+
+    def step():
+        rk.gather(ids.data_ptr(), n, x.data_ptr(), xg.data_ptr(), ssp.data_ptr())
+
+    for _ in range(args.warmup):
+        step()
+    rk.sync()
+    props = torch.cuda.get_device_properties(local_rank)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local_rank)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_id) as clk:
+        torch.cuda.synchronize()
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize()
+    rk.sync()
+    ms = start.elapsed_time(end) / args.steps
+    pk = peaks()
+    bytes_per = 2 * d + 4 * d + 2 * d + 4 * (d // 64)  # fp16 row read; fp32 x, fp16 x g, sums written
+    gbs = n * bytes_per / (ms / 1e3) / 1e9
+    if rank == 0:
+        print(json.dumps({
+            "metric": "VID gather lookups/s (standalone, Zipf(1.1) over a 1M-row FP16 table)",
+            "value": n / (ms / 1e3), "unit": "lookups/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "config": {"workload": f"gather: {n} lookups, Zipf(1.1) over {GATHER_TABLE_ROWS} rows x {d} fp16",
+                       "bytes_per_lookup": bytes_per, "l2": "no flush: 2 GB table, 27 GB written per step"},
+            "e2e": None,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm"], "traffic": None,
+                         "kernel": "embed_gain_kernel (through duolm_gather)",
+                         "peak_note": f"{pk['src']} copy bandwidth"},
+            "gpu_launches": args.steps,
+            "clocks": clk.summary(),
+            "cpu_baseline": None,
+        }), flush=True)
+    rk.close()
 
 
 def run_ours(args, rank: int, world: int, local_rank: int) -> None:
@@ -410,9 +486,13 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu:
         per, nc = oracle_time(wl, [0])
+        per_i, nc_i = oracle_time(wl, [0], independent_cands=4)
         cpu = {"value": nc / sum(per), "unit": UNIT, "cores": cpu_count(), "kind": "oracle",
                "sample": f"request 0 of the {wl.name} batch (L={wl.requests[0].L}, K={wl.requests[0].K}) "
-                         f"through the oracle's packed layout, {sum(per):.1f} s"}
+                         f"through the oracle's packed layout, {sum(per):.1f} s",
+               "independent": {"value": nc_i / sum(per_i), "unit": UNIT,
+                               "sample": f"4 candidates of request 0 scored independently (each its own "
+                                         f"L + b sequence), {sum(per_i):.1f} s"}}
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -459,6 +539,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+    elif args.config == "gather":
+        run_gather(args, rank, world, local_rank)
     else:
         run_ours(args, rank, world, local_rank)
 

@@ -170,6 +170,30 @@ const char *duolm_last_error(const duolm_ctx *ctx);
 /* Free every device resource of the context (NULL is ignored). */
 void duolm_destroy(duolm_ctx *ctx);
 
+/*
+ * duolm_gather -- the hot path's first step alone: the virtual-id gather of
+ * the ranker's inputs (DuoLM summary page, 方法步骤详情 step 3: an id below
+ * the vocabulary V reads the embedding, id V + i reads row i of the FP16 item
+ * table) with what the gather writes for the first layer's norm, for n ids
+ * already in device memory.  Lets the gather be measured on its own (for
+ * example over millions of lookups of a large table) and checked row by row.
+ *   ids:  device int32 [n], each in [0, V + n_items); read only.  An id out of
+ *         range raises the device error flag (reported by the next
+ *         duolm_sync as DUOLM_E_DEVICE) and its row is written as zeros.
+ *   x:    device float [n][d]: the gathered rows (fp32; the fp16 table and
+ *         bf16 embedding values are exact in fp32).
+ *   xg:   device uint16 [n][d]: fp16 bit patterns of x times the first
+ *         layer's attention-norm gain.
+ *   ssp:  device float [n][d / 64]: per row, slot 0 holds the sum of x^2 and
+ *         the other slots 0.
+ * All buffers belong to the caller.  The work is queued on the context's
+ * stream and the call returns without waiting (duolm_sync waits and checks
+ * the error flag).  Returns DUOLM_E_ARG for n < 0, n > INT32_MAX or a null
+ * pointer with n > 0; DUOLM_E_STATE for an fp32 model (its gather normalises
+ * in place instead).
+ */
+int duolm_gather(duolm_ctx *ctx, const int32_t *ids, int64_t n, float *x, uint16_t *xg, float *ssp);
+
 /* Largest vocabulary duolm_embedding_rho_static accepts (rows of its
  * built-in scratch array: 2 MB of fp64, held by every GPU that loads the
  * library until the process exits). */

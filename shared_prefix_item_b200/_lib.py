@@ -67,6 +67,7 @@ def _load():
         "duolm_profile": (I, [VP, I, VP, VP]),
         "duolm_debug_wait_timeout": (I, [VP]),
         "duolm_embedding_rho_static": (I, [VP, I, I64, I, VP, VP]),
+        "duolm_gather": (I, [VP, VP, I64, VP, VP, VP]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -210,6 +211,12 @@ class Ranker:
         out = np.empty((tq, tq), np.uint8)
         self._check(lib.duolm_debug_mask(self.ctx, int(request), _p(out)))
         return out.astype(bool)
+
+    def gather(self, ids_dev: int, n: int, x_dev: int, xg_dev: int, ssp_dev: int) -> None:
+        """duolm_gather: the VID gather alone on device buffers (queued on the
+        context's stream; sync() waits and checks the error flag)."""
+        self._check(lib.duolm_gather(self.ctx, ctypes.c_void_p(ids_dev), int(n), ctypes.c_void_p(x_dev),
+                                     ctypes.c_void_p(xg_dev), ctypes.c_void_p(ssp_dev)))
 
     def debug_residual(self, n_layers: int, n_tokens: int) -> np.ndarray:
         out = np.empty((n_tokens, self.d), np.float32)

@@ -67,6 +67,7 @@ struct duolm_ctx {
   float2* rope = nullptr;
   DevStatus* status = nullptr;
   double* rho_buf = nullptr;
+  PlanHdr* gather_hdr = nullptr;  // header through which duolm_gather hands the caller's ids to the gather
 
   int64_t cap_T = 0, cap_R = 0, cap_C = 0, cap_I = 0, plan_cap = 0;
   float* x = nullptr;
@@ -896,6 +897,7 @@ void duolm_destroy(duolm_ctx* ctx) {
   dfree(ctx->rope);
   dfree(ctx->status);
   dfree(ctx->rho_buf);
+  dfree(ctx->gather_hdr);
   if (ctx->plan_ev) cudaEventDestroy(ctx->plan_ev);
   if (ctx->own_stream && ctx->stream) cudaStreamDestroy(ctx->stream);
   delete ctx;
@@ -974,6 +976,28 @@ int duolm_debug_gemm(duolm_ctx* ctx, int layer, int which, const uint16_t* a, fl
   cudaFree(tmp);
   if (e != cudaSuccess) return fail(ctx, DUOLM_E_CUDA, "debug_gemm: %s", cudaGetErrorString(e));
   return check_status(ctx);
+}
+
+int duolm_gather(duolm_ctx* ctx, const int32_t* ids, int64_t n, float* x, uint16_t* xg, float* ssp) {
+  if (!ctx || n < 0 || n > INT32_MAX || (n > 0 && (!ids || !x || !xg || !ssp)))
+    return fail(ctx, DUOLM_E_ARG, "gather: bad arguments");
+  if (!ctx->f16) return fail(ctx, DUOLM_E_STATE, "gather: only bf16 models run the fp16 gather");
+  if (n == 0) return 0;
+  CK(cudaSetDevice(ctx->device));
+  if (!ctx->gather_hdr)
+    if (int rc = dalloc(ctx, &ctx->gather_hdr, sizeof(PlanHdr))) return rc;
+  // the kernel finds its ids at a byte offset from the header: point it at
+  // the caller's array (the header is staged from host memory before the
+  // copy call returns, so a stack copy is fine)
+  PlanHdr h{};
+  h.n_tokens = (int32_t)n;
+  h.off_ids = (int64_t)(reinterpret_cast<const char*>(ids) - reinterpret_cast<const char*>(ctx->gather_hdr));
+  CK(cudaMemcpyAsync(ctx->gather_hdr, &h, sizeof h, cudaMemcpyHostToDevice, ctx->stream));
+  const duolm_model_desc& d = ctx->desc;
+  CK(embed_gain(ctx->gather_hdr, ctx->embed, ctx->table, ctx->n_items, d.vocab, d.d,
+                ctx->gains + ctx->layers[0].g_attn, x, reinterpret_cast<__half*>(xg), ssp, d.d / 64, ctx->status,
+                (int)std::min<int64_t>(n, INT32_MAX), ctx->stream));
+  return 0;
 }
 
 int duolm_debug_wait_timeout(duolm_ctx* ctx) {

@@ -186,6 +186,17 @@ def _zipf_sampler(n_items: int, s_exp: float):
     return draw
 
 
+def zipf_lookups(n: int, n_items: int = 1_000_000, s_exp: float = 1.1, seed: int = SEED_REQUESTS + 5) -> np.ndarray:
+    """n item-table row indices drawn Zipf(s_exp) over n_items rows, with
+    replacement: the stream of VID reads that many requests' histories and
+    candidates produce on a large catalog (popular items recur)."""
+    ranks = np.arange(1, n_items + 1, dtype=np.float64)
+    cdf = np.cumsum(ranks ** -s_exp)
+    cdf /= cdf[-1]
+    u = Stream(seed, 0).uniform(n)
+    return np.minimum(np.searchsorted(cdf, u, side="right"), n_items - 1).astype(np.int64)
+
+
 def make_request(s: Stream, tpl: _Template, vocab: int, n_items: int, n_hist: int,
                  feedback_lens, n_cand: int, branch_len: int, item_draw=None,
                  random_branch_header: bool = False) -> Request:

@@ -95,3 +95,4 @@ def test_reference_arm_other_ranks_do_no_work(capsys):
             raise AssertionError(f"rank 1 read --{k}")
     bench.run_reference(Args(), 1, 2)
     assert capsys.readouterr().out == ""
+
