@@ -48,6 +48,8 @@ def workload(name: str, shard: int) -> W.Workload:
         return W.c1(shard=shard)
     if name == "stress":
         return W.stress(shard=shard)
+    if name.startswith("fir-m"):
+        return W.fir(int(name[len("fir-m"):]), shard=shard)
     if name.startswith("catalog-c"):
         return W.catalog(int(name[len("catalog-c"):]), shard=shard)
     raise SystemExit(f"unknown config {name}")
@@ -300,6 +302,24 @@ def run_reference(args, rank: int, world: int) -> None:
     print(json.dumps(line), flush=True)
 
 
+TABLE_BUILD_ROWS = 100_000
+
+
+def load_table(rk, n_rows: int, d: int) -> str:
+    """The item table of a workload: built through the library's interface
+    kernel from the seeded item vectors; above TABLE_BUILD_ROWS rows the first
+    TABLE_BUILD_ROWS are built and tiled (the values do not affect the
+    timing, and generating millions of vectors on the host takes minutes).
+    Returns a note for the config."""
+    base = min(n_rows, TABLE_BUILD_ROWS)
+    rk.vid_table_build(W.item_vectors(base, d), 0.0, rk.embedding_rho())
+    if base == n_rows:
+        return f"{n_rows} rows from the seeded item vectors"
+    reps = -(-n_rows // base)
+    rk.vid_table_load(np.tile(rk.debug_table(base), (reps, 1))[:n_rows])
+    return f"{n_rows} rows: {base} from the seeded item vectors, tiled"
+
+
 GATHER_LOOKUPS = 4_194_304
 GATHER_TABLE_ROWS = 1_000_000
 
@@ -316,14 +336,7 @@ def run_gather(args, rank: int, world: int, local_rank: int) -> None:
     stream = torch.cuda.Stream()
     torch.cuda.set_stream(stream)
     rk = S.Ranker(shape, W.model_weights(shape), device=local_rank, stream=stream.cuda_stream)
-    # a 1M-row table: 10k rows through the library's own interface, tiled
-    # (the values do not matter to the measurement, the size and the access
-    # pattern do)
-    base_rows = 10_000
-    rk.vid_table_build(W.item_vectors(base_rows, shape.d), 0.0, rk.embedding_rho())
-    rows = np.tile(rk.debug_table(base_rows), (GATHER_TABLE_ROWS // base_rows, 1))
-    rk.vid_table_load(rows)
-    del rows
+    load_table(rk, GATHER_TABLE_ROWS, shape.d)
     n, d = GATHER_LOOKUPS, shape.d
     ids = torch.from_numpy((shape.vocab + W.zipf_lookups(n, GATHER_TABLE_ROWS)).astype(np.int32)).cuda()
     x = torch.empty((n, d), dtype=torch.float32, device="cuda")
@@ -391,7 +404,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     stream = torch.cuda.Stream()
     torch.cuda.set_stream(stream)
     rk = S.Ranker(shape, W.model_weights(shape), device=local_rank, stream=stream.cuda_stream)
-    rk.vid_table_build(W.item_vectors(wl.n_items, shape.d), 0.0, rk.embedding_rho())
+    table_note = load_table(rk, wl.n_items, shape.d)
     rk.set_graph(not args.no_graph)
     p, po, b, co = wl.packed()
     rk.prepare(p, po, b, co, wl.branch_len, mode)
@@ -499,7 +512,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": value / H100_C64 if args.config == "c64" and not indep else None,
             "dtype": "f16", "data": "synthetic",
-            "config": describe(wl, args.mode, not args.no_graph, world),
+            "config": {**describe(wl, args.mode, not args.no_graph, world), "table": table_note},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4 * n_cand},
             "roofline": dominant,
             "roofline_step": {"flops_per_step": gf + af, "ms_at_peak": step_roof_ms,

@@ -220,6 +220,51 @@ def make_request(s: Stream, tpl: _Template, vocab: int, n_items: int, n_hist: in
     return Request(prefix, branch.astype(np.int32), hist, cands)
 
 
+def make_mv_request(s: Stream, tpl: _Template, vocab: int, n_items: int, m: int, n_hist: int, feedback_lens,
+                    n_cand: int) -> Request:
+    """A request over multi-vector items: item i is the m table rows i m ..
+    i m + m - 1 (ids V + i m + k).  A history item is the marker followed by
+    its m VIDs and its feedback tokens; a candidate branch is its m VIDs (b = m),
+    scored at the last one."""
+    hist = s.distinct(n_hist, 0, n_items)
+    cands = s.distinct(n_cand, 0, n_items, hist)
+    parts = [tpl.instr]
+    for i, it in enumerate(hist):
+        fb = s.integers(int(feedback_lens[i]), 0, vocab)
+        parts += [np.array([tpl.marker]), vocab + it * m + np.arange(m), fb]
+    parts.append(tpl.header)
+    prefix = np.concatenate([np.asarray(p, np.int64) for p in parts]).astype(np.int32)
+    branch = vocab + cands[:, None] * m + np.arange(m)[None, :]
+    return Request(prefix, branch.astype(np.int32), hist, cands)
+
+
+def fir(m: int = 8, n_requests: int = 64, shard: int = 0) -> Workload:
+    """The 64-request recipe with multi-vector items of m rows each: history
+    U{1..20} items, U{8..48} feedback tokens per item, K = 100 candidates of
+    m tokens, 100k items = 100k m table rows."""
+    model = QWEN3_06B
+    n_items = 100_000
+    s = Stream(SEED_REQUESTS + 6, shard)
+    tpl = _Template(s, model.vocab, 32, 4, 0)
+    reqs = []
+    for _ in range(n_requests):
+        h = int(s.integers(1, 1, 21)[0])
+        f = s.integers(h, 8, 49)
+        reqs.append(make_mv_request(s, tpl, model.vocab, n_items, m, h, f, 100))
+    return Workload(f"fir-m{m}", model, n_items * m, m, reqs)
+
+
+def custom_fir(model: ModelShape, n_items: int, seed: int, n_requests: int, n_hist: int, feedback: int,
+               n_cand: int, m: int) -> Workload:
+    """Small multi-vector workloads for parity tests (n_items items, n_items m
+    table rows)."""
+    s = Stream(seed, 11)
+    tpl = _Template(s, model.vocab, 3, 2, 0)
+    reqs = [make_mv_request(s, tpl, model.vocab, n_items, m, n_hist, [feedback] * n_hist, n_cand)
+            for _ in range(n_requests)]
+    return Workload(f"custom-fir-m{m}", model, n_items * m, m, reqs)
+
+
 def tiny(seed_offset: int = 0) -> Workload:
     """Tiny fp32 ranker, one request: L = 8 + 4 x (1 + 1 + 8) = 48, K = 8, b = 1."""
     m = TINY

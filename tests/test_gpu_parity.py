@@ -155,6 +155,22 @@ def test_q2_ragged_scores(seed, n_req, n_hist, fb, K, b, n_instr):
         P.assert_scores_match(Q2, got_ind[q], ref, f"req {q} independent")
 
 
+def test_q2_multivector_items():
+    # items of m = 8 table rows: a history item is the marker and its 8 VIDs,
+    # a candidate branch is its 8 VIDs (b = 8), scored at the last one
+    wl = W.custom_fir(Q2, Q2_ITEMS // 8, 901, 2, 3, 6, 12, 8)
+    assert wl.n_items == Q2_ITEMS
+    rk = P.ranker(Q2, Q2_ITEMS)
+    otab = P.oracle_table(Q2, Q2_ITEMS)[0]
+    om = P.oracle_model(Q2)
+    got = P.split_scores(wl, rk.score_workload(wl))
+    got_ind = P.split_scores(wl, rk.score_workload(wl, 1))
+    for q, r in enumerate(wl.requests):
+        ref = R.score_mis(om, otab, r)
+        P.assert_scores_match(Q2, got[q], ref, f"req {q}")
+        P.assert_scores_match(Q2, got_ind[q], ref, f"req {q} independent")
+
+
 def test_graph_replay_matches_eager_and_is_deterministic():
     wl = W.custom(Q2, Q2_ITEMS, 321, 3, (1, 6), (3, 20), (5, 40), 1, n_instr=7)
     rk = P.ranker(Q2, Q2_ITEMS)
