@@ -384,6 +384,55 @@ def run_gather(args, rank: int, world: int, local_rank: int) -> None:
     rk.close()
 
 
+LATENCY_CALLS = {1: 200, 8: 100, 64: 40}
+
+
+def run_latency(args, rank: int, world: int, local_rank: int) -> None:
+    """Closed-loop latency of the public call: for C in {1, 8, 64}, each call
+    scores a fresh batch of C requests of the 64-request recipe from host
+    buffers (duolm_score: validation, packing, host->device plan copy, the
+    pass, scores back), timed on the host clock around the blocking call;
+    p50/p99 over the calls, with the CUDA graph on and off.  A request's
+    latency is its call's (no queueing: one call at a time)."""
+    import torch
+
+    import shared_prefix_item_b200 as S
+    torch.cuda.set_device(local_rank)
+    shape = W.QWEN3_06B
+    rk = S.Ranker(shape, W.model_weights(shape), device=local_rank)
+    table_note = load_table(rk, 100_000, shape.d)
+    out = {}
+    for C, n_calls in LATENCY_CALLS.items():
+        batches = [W.c64(n_requests=C, shard=1000 + i).packed() for i in range(n_calls)]
+        rk.reserve(max(int(len(b[0]) + len(b[2])) for b in batches), C, C * 100)
+        res = {}
+        for graph in (True, False):
+            rk.set_graph(graph)
+            for b in batches[:3]:  # warm-up (graph capture at this capacity)
+                rk.score(b[0], b[1], b[2], b[3], 1)
+            t = []
+            for b in batches:
+                t0 = time.perf_counter()
+                rk.score(b[0], b[1], b[2], b[3], 1)
+                t.append((time.perf_counter() - t0) * 1e3)
+            t = np.array(t)
+            res["graph" if graph else "eager"] = {"p50_ms": float(np.percentile(t, 50)),
+                                                  "p99_ms": float(np.percentile(t, 99)),
+                                                  "mean_ms": float(t.mean()), "calls": n_calls}
+        out[f"C={C}"] = res
+    if rank == 0:
+        print(json.dumps({
+            "metric": "per-call latency of duolm_score, closed loop (p99, C=64, graph)",
+            "value": out["C=64"]["graph"]["p99_ms"], "unit": "ms", "n_gpus": 1, "steps": None,
+            "warmup": 3, "higher_is_better": False, "scaling": None, "vs_baseline": None, "dtype": "f16",
+            "data": "synthetic",
+            "config": {"workload": "fresh batches of C requests of the 64-request recipe (K=100, b=1) per call",
+                       "table": table_note, "timing": "host clock around the blocking call"},
+            "latency": out,
+        }), flush=True)
+    rk.close()
+
+
 def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     import torch
 
@@ -554,6 +603,8 @@ def main():
         run_reference(args, rank, world)
     elif args.config == "gather":
         run_gather(args, rank, world, local_rank)
+    elif args.config == "latency":
+        run_latency(args, rank, world, local_rank)
     else:
         run_ours(args, rank, world, local_rank)
 
