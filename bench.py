@@ -38,7 +38,8 @@ from synth import workloads as W  # noqa: E402
 
 METRIC = "candidate scores/sec on 1 B200 (Qwen3-0.6B shape, K=100) + % of roofline"
 UNIT = "candidate scores/s"
-H100_C64 = 26404.0  # pages' figure: MIS + CUDA Graph, C=64, 100 candidates, 1x H100 (context)
+# the pages' figures for this metric (1x H100, 100 candidates per request; context, not targets)
+PAGES_CAND_PER_S = {("c64", "mis"): 26404.0, ("c1", "mis"): 8870.0, ("c64", "independent"): 851.48}
 
 
 def workload(name: str, shard: int) -> W.Workload:
@@ -559,7 +560,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": value / H100_C64 if args.config == "c64" and not indep else None,
+            "vs_baseline": (value / PAGES_CAND_PER_S[(args.config, args.mode)]
+                            if (args.config, args.mode) in PAGES_CAND_PER_S else None),
             "dtype": "f16", "data": "synthetic",
             "config": {**describe(wl, args.mode, not args.no_graph, world), "table": table_note},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4 * n_cand},
