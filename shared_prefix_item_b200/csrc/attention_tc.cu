@@ -95,7 +95,10 @@ __device__ __forceinline__ Item make_item(int4 item, int4 rq, int b) {
 }
 
 // Work-list reader that keeps the descriptors of the next two items in
-// flight, so a role never waits on global memory at an item boundary.
+// flight, so a role never waits on global memory at an item boundary.  A
+// CTA runs the contiguous range of the work list the plan gives it (the
+// host's load-balanced schedule), or, for a plan divided among a different
+// number of CTAs, every gridDim.x-th item.
 template <int G>
 struct ItemStream {
   const int4* items;
@@ -103,9 +106,18 @@ struct ItemStream {
   int n, step, b;
   int it;
   int4 d1, d2, r1;  // descriptor of it + step, it + 2 step; request of it + step
-  __device__ ItemStream(const PlanHdr* plan, int first, int step_, int b_)
-      : items(plan_array<int4>(plan, plan->off_items)), reqs(plan_array<int4>(plan, plan->off_req)),
-        n(plan->n_items), step(step_), b(b_), it(first) {
+  __device__ ItemStream(const PlanHdr* plan, int cta, int n_ctas, int b_)
+      : items(plan_array<int4>(plan, plan->off_items)), reqs(plan_array<int4>(plan, plan->off_req)), b(b_) {
+    if (plan->att_ctas == n_ctas) {
+      const int32_t* off = plan_array<int32_t>(plan, plan->off_cta);
+      it = off[cta];
+      n = off[cta + 1];
+      step = 1;
+    } else {
+      it = cta;
+      n = plan->n_items;
+      step = n_ctas;
+    }
     const int4 z = make_int4(0, 0, 0, 0);
     d1 = it < n ? items[it] : z;
     d2 = it + step < n ? items[it + step] : z;

@@ -43,14 +43,16 @@ struct PlanHdr {
   int32_t n_cand;       // scored candidates
   int32_t branch_len;   // b
   int32_t n_items;      // attention work items
-  int32_t pad0, pad1, pad2;
+  int32_t att_ctas;     // CTAs the attention work list is divided among (0: none)
+  int32_t pad1, pad2;
   int64_t off_ids;      // int32 [T]   ranker ids
   int64_t off_pos;      // int32 [T]   position ids
   int64_t off_req;      // int4  [n_req]  {tok0, L, K, 0}
   int64_t off_cand;     // int32 [n_cand] packed row of each candidate's last token
   int64_t off_items;    // int4  [n_items] {req, kv_head, kind, row0}
   int64_t off_treq;     // int32 [T]   request of each token
-  int64_t pad4, pad5;
+  int64_t off_cta;      // int32 [att_ctas + 1] items of CTA c: [off_cta[c], off_cta[c + 1])
+  int64_t pad5;
 };
 static_assert(sizeof(PlanHdr) == 96, "plan header layout");
 

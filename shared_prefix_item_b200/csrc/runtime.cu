@@ -13,6 +13,7 @@
 #include <cstring>
 #include <string>
 #include <thread>
+#include <queue>
 #include <vector>
 
 #include "common.cuh"
@@ -246,8 +247,9 @@ int64_t items_bound(const duolm_ctx* c, int64_t T, int64_t R) {
   return (int64_t)c->desc.n_kv_heads * (2 * T / r + 2 * R + 2);
 }
 
-int64_t plan_bytes_for(int64_t T, int64_t R, int64_t C, int64_t I) {
-  return (int64_t)sizeof(PlanHdr) + 3 * align16(T * 4) + align16(R * 16) + align16(C * 4) + align16(I * 16);
+int64_t plan_bytes_for(int64_t T, int64_t R, int64_t C, int64_t I, int64_t G) {
+  return (int64_t)sizeof(PlanHdr) + 3 * align16(T * 4) + align16(R * 16) + align16(C * 4) + align16(I * 16) +
+         align16((G + 1) * 4);
 }
 
 int reserve_impl(duolm_ctx* ctx, int64_t T, int64_t R, int64_t C) {
@@ -284,7 +286,7 @@ int reserve_impl(duolm_ctx* ctx, int64_t T, int64_t R, int64_t C) {
   }
   if ((rc = dalloc(ctx, &ctx->scores, C * 4))) return rc;
   const int64_t I = items_bound(ctx, T, R);
-  const int64_t pb = plan_bytes_for(T, R, C, I);
+  const int64_t pb = plan_bytes_for(T, R, C, I, ctx->num_sms);
   if ((rc = dalloc(ctx, &ctx->plan_dev, pb))) return rc;
   CK(cudaMallocHost(reinterpret_cast<void**>(&ctx->plan_host), pb));
   ctx->cap_T = T;
@@ -759,9 +761,45 @@ int duolm_prepare(duolm_ctx* ctx, int n_requests, const int32_t* prefix_ids, con
       for (int row0 = 0; row0 < K * branch_len; row0 += per) it[n_items++] = int4{r, kvh, 1, row0};
       for (int row0 = ((L - 1) / Rw) * Rw; row0 >= 0; row0 -= Rw) it[n_items++] = int4{r, kvh, 0, row0};
     }
+    // Each CTA runs the items the greedy list schedule gives it: in list
+    // order, an item goes to the CTA with the least work so far.  The
+    // estimated cost of an item is its key tiles, +20% when its second
+    // query sub-tile is in use (the two sub-tiles run side by side), plus
+    // half a tile for starting it.  Items stay in list order within a CTA and
+    // CTAs advance through the list at about the same pace, so the items of
+    // one (request, KV head) still run close together in time.
+    const int G = ctx->num_sms;
+    std::vector<int> owner((size_t)n_items);
+    {
+      std::priority_queue<std::pair<int64_t, int>, std::vector<std::pair<int64_t, int>>, std::greater<>> load;
+      for (int g = 0; g < G; ++g) load.push({0, g});
+      const int half_rows = Rw / 2;  // rows of one query sub-tile
+      for (int64_t i = 0; i < n_items; ++i) {
+        const int4 m = it[i];
+        const int L = rq[m.x].y, K = rq[m.x].z;
+        const int nrows = m.z ? std::min(per, K * branch_len - m.w) : std::min(Rw, L - m.w);
+        const int kend = m.z ? L : std::min(m.w + Rw, L);
+        const int64_t tiles = (kend + key_tile - 1) / key_tile + (m.z ? (nrows + key_tile - 1) / key_tile : 0);
+        const int64_t cost = 10 * tiles + (nrows > half_rows ? 2 * tiles : 0) + 5;
+        auto top = load.top();
+        load.pop();
+        owner[i] = top.second;
+        load.push({top.first + cost, top.second});
+      }
+    }
+    std::vector<int4> listed(it, it + n_items);
+    hdr.att_ctas = G;
+    hdr.off_cta = hdr.off_items + align16(n_items * 16);
+    int32_t* cta_off = reinterpret_cast<int32_t*>(base + hdr.off_cta);
+    std::fill(cta_off, cta_off + G + 1, 0);
+    for (int64_t i = 0; i < n_items; ++i) ++cta_off[owner[i] + 1];
+    for (int g = 0; g < G; ++g) cta_off[g + 1] += cta_off[g];
+    std::vector<int32_t> fill(cta_off, cta_off + G);
+    for (int64_t i = 0; i < n_items; ++i) it[fill[owner[i]]++] = listed[i];
   }
   hdr.n_items = (int32_t)n_items;
-  const int64_t bytes = hdr.off_items + align16(n_items * 16);
+  const int64_t bytes = hdr.att_ctas ? hdr.off_cta + align16((int64_t)(hdr.att_ctas + 1) * 4)
+                                     : hdr.off_items + align16(n_items * 16);
   memcpy(base, &hdr, sizeof hdr);
   CK(cudaMemcpyAsync(ctx->plan_dev, base, bytes, cudaMemcpyHostToDevice, ctx->stream));
   CK(cudaEventRecord(ctx->plan_ev, ctx->stream));
@@ -946,7 +984,8 @@ int duolm_debug_residual(duolm_ctx* ctx, int n_layers, float* x_out) {
 
 int64_t duolm_plan_bytes(const duolm_ctx* ctx) {
   if (!ctx || !ctx->prepared) return 0;
-  return ctx->hdr.off_items + align16((int64_t)ctx->hdr.n_items * 16);
+  return ctx->hdr.att_ctas ? ctx->hdr.off_cta + align16((int64_t)(ctx->hdr.att_ctas + 1) * 4)
+                           : ctx->hdr.off_items + align16((int64_t)ctx->hdr.n_items * 16);
 }
 
 int duolm_debug_gemm(duolm_ctx* ctx, int layer, int which, const uint16_t* a, float* out) {
