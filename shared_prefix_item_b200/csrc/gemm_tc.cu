@@ -84,14 +84,11 @@ __device__ __forceinline__ float row_rnorm(const float* ssp, int n_slots, int ro
 // 16-byte-aligned destination of row r of the warp, or null to skip it.
 constexpr int kScratchPad = 36;
 constexpr int kScratchPerWarp = 32 * kScratchPad * 4;
+// The second half of that: the scratch already holds the warp's 32 rows.
 template <class Dst>
-__device__ __forceinline__ void warp_store_rows_128B(uint32_t* buf, const uint32_t (&v)[32], Dst dst) {
+__device__ __forceinline__ void warp_flush_rows_128B(const uint32_t* buf, Dst dst) {
   const int lane = threadIdx.x & 31;
-  __syncwarp();  // earlier reads of the scratch are done
-#pragma unroll
-  for (int q = 0; q < 8; ++q)
-    *reinterpret_cast<uint4*>(buf + lane * kScratchPad + 4 * q) = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-  __syncwarp();
+  __syncwarp();  // every lane's writes to the scratch are done
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int r = 4 * i + (lane >> 3);
@@ -99,6 +96,15 @@ __device__ __forceinline__ void warp_store_rows_128B(uint32_t* buf, const uint32
     uint4* p = dst(r);
     if (p) p[lane & 7] = w;
   }
+}
+template <class Dst>
+__device__ __forceinline__ void warp_store_rows_128B(uint32_t* buf, const uint32_t (&v)[32], Dst dst) {
+  const int lane = threadIdx.x & 31;
+  __syncwarp();  // earlier reads of the scratch are done
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    *reinterpret_cast<uint4*>(buf + lane * kScratchPad + 4 * q) = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  warp_flush_rows_128B(buf, dst);
 }
 
 struct EpiResid {
@@ -244,8 +250,11 @@ struct EpiSwiglu {
 struct EpiQkv {
   EpiQkvArgs a;
   static constexpr int EG = 2;  // one head of the 256-column tile per group
-  static constexpr int STAGES = 6;
-  static constexpr int SCRATCH_PER_WARP = 0;
+  // rows leave through two per-warp scratches (the head's two 64-column
+  // halves), four full lines per warp store; a 4-stage ring keeps the CTA
+  // near 200 KB
+  static constexpr int STAGES = 4;
+  static constexpr int SCRATCH_PER_WARP = 2 * kScratchPerWarp;
   struct Pre {};
   template <int BN>
   __device__ __forceinline__ Pre prefetch(int, int, int, bool, const PlanHdr*, DevStatus*) const {
@@ -253,38 +262,46 @@ struct EpiQkv {
   }
   template <int BN>
   __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, int g, bool row_ok, const PlanHdr* plan,
-                                      DevStatus* st, uint8_t*, int, const Pre&) const {
+                                      DevStatus* st, uint8_t* scratch, int M, const Pre&) const {
     const int gc = n0 + 128 * g;
     const uint32_t base = taddr + 128 * g;
+    const int lane = threadIdx.x & 31;
+    const int row0 = row - lane;
+    uint32_t* buf1 = reinterpret_cast<uint32_t*>(scratch);
+    uint32_t* buf2 = buf1 + 32 * kScratchPad;
     // weight scale times the input row's RMSNorm factor
     const float sc = row_ok ? a.scale * row_rnorm(a.ssp, a.n_slots, row, a.inv_d, a.norm_eps) : 0.f;
     if (gc >= a.qd + a.kd) {  // value head
       const int head = (gc - a.qd - a.kd) >> 7;
-      __half* dst = a.vc + ((int64_t)head * a.kv_rows + row) * 128;
 #pragma unroll 1
-      for (int c = 0; c < 128; c += 16) {
-        float v[16];
-        tmem_ld16(base + c, v);
-        if (row_ok) {
-          uint32_t pk[8];
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            __half2 hh = __halves2half2(to_half_checked(v[2 * j] * sc, st, 21),
-                                        to_half_checked(v[2 * j + 1] * sc, st, 21));
-            pk[j] = *reinterpret_cast<uint32_t*>(&hh);
+        for (int q = 0; q < 2; ++q) {
+          float v[32];
+          tmem_ld32(base + 64 * half + 32 * q, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            __half2 hh = row_ok ? __halves2half2(to_half_checked(v[2 * j] * sc, st, 21),
+                                                 to_half_checked(v[2 * j + 1] * sc, st, 21))
+                                : __halves2half2(__float2half_rn(0.f), __float2half_rn(0.f));
+            pk[16 * q + j] = *reinterpret_cast<uint32_t*>(&hh);
           }
-          uint4* p = reinterpret_cast<uint4*>(dst + c);
-          p[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          p[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
+        warp_store_rows_128B(buf1, pk, [&](int r) -> uint4* {
+          const int rr = row0 + r;
+          return rr < M ? reinterpret_cast<uint4*>(a.vc + ((int64_t)head * a.kv_rows + rr) * 128 + 64 * half)
+                        : nullptr;
+        });
       }
       return;
     }
     const bool is_q = gc < a.qd;
     const int head = is_q ? (gc >> 7) : ((gc - a.qd) >> 7);
     const float* gain = is_q ? a.gq : a.gk;
-    __half* dst = is_q ? a.q + ((int64_t)row * a.n_q_heads + head) * 128
-                       : a.kc + ((int64_t)head * a.kv_rows + row) * 128;
+    auto dst = [&](int rr) -> __half* {
+      return is_q ? a.q + ((int64_t)rr * a.n_q_heads + head) * 128 : a.kc + ((int64_t)head * a.kv_rows + rr) * 128;
+    };
     float ss = 0.f;
 #pragma unroll 1
     for (int c = 0; c < 128; c += 16) {
@@ -306,6 +323,7 @@ struct EpiQkv {
       }
     }
     const float2* cs = a.rope + p;  // entry (i, p) at cs[i * max_pos]
+    __syncwarp();  // the previous tile's reads of the scratches are done
 #pragma unroll 1
     for (int c = 0; c < 64; c += 16) {
       float x1[16], x2[16];
@@ -341,14 +359,23 @@ struct EpiQkv {
           o1[j / 2] = *reinterpret_cast<uint32_t*>(&h1);
           o2[j / 2] = *reinterpret_cast<uint32_t*>(&h2);
         }
-        uint4* p1 = reinterpret_cast<uint4*>(dst + c);
-        uint4* p2 = reinterpret_cast<uint4*>(dst + 64 + c);
-        p1[0] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
-        p1[1] = make_uint4(o1[4], o1[5], o1[6], o1[7]);
-        p2[0] = make_uint4(o2[0], o2[1], o2[2], o2[3]);
-        p2[1] = make_uint4(o2[4], o2[5], o2[6], o2[7]);
+        // this chunk's 16 + 16 outputs into the row's slots of the scratches
+        uint32_t* s1 = buf1 + lane * kScratchPad + c / 2;
+        uint32_t* s2 = buf2 + lane * kScratchPad + c / 2;
+        reinterpret_cast<uint4*>(s1)[0] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+        reinterpret_cast<uint4*>(s1)[1] = make_uint4(o1[4], o1[5], o1[6], o1[7]);
+        reinterpret_cast<uint4*>(s2)[0] = make_uint4(o2[0], o2[1], o2[2], o2[3]);
+        reinterpret_cast<uint4*>(s2)[1] = make_uint4(o2[4], o2[5], o2[6], o2[7]);
       }
     }
+    warp_flush_rows_128B(buf1, [&](int r) -> uint4* {
+      const int rr = row0 + r;
+      return rr < M ? reinterpret_cast<uint4*>(dst(rr)) : nullptr;
+    });
+    warp_flush_rows_128B(buf2, [&](int r) -> uint4* {
+      const int rr = row0 + r;
+      return rr < M ? reinterpret_cast<uint4*>(dst(rr) + 64) : nullptr;
+    });
   }
 };
 
