@@ -131,12 +131,21 @@ KERNEL_SOURCES = {  # the files a kernel class is built from (its ncu traffic is
 }
 
 
+def code_text(src: str) -> str:
+    """The code of a C++/CUDA source without its comments and with
+    whitespace collapsed (an edit to a comment does not change a kernel)."""
+    import re
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
+
+
 def source_hash(kind: str) -> str:
     import hashlib
     h = hashlib.sha256()
     for f in KERNEL_SOURCES[kind]:
-        with open(os.path.join(ROOT, "shared_prefix_item_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "shared_prefix_item_b200", "csrc", f), encoding="utf-8") as fh:
+            h.update(code_text(fh.read()).encode())
     return h.hexdigest()[:16]
 
 
