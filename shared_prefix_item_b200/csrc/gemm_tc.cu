@@ -1,15 +1,21 @@
 // Projection GEMMs of the ranker on 5th-generation tensor cores (sm_100a).
 //
 // C[M, N] = A[M, K] * B[N, K]^T with fp16 operands and fp32 accumulation in
-// tensor memory.  One persistent CTA per SM, warp-specialised:
-//   warp 0      TMA producer: streams 128x64 A and BNx64 B tiles (128-byte
-//               swizzle, no multicast) into a STAGES-deep shared-memory ring;
-//   warp 1      allocates 2*BN TMEM columns; lane 0 issues tcgen05.mma
-//               (128 x BN x 16 per instruction) and commits to mbarriers;
+// tensor memory.  Persistent clusters of two CTAs (one per SM), each pair
+// computing 256 x BN tiles, warp-specialised per CTA:
+//   warp 0      TMA producer: streams this CTA's 128x64 A block and its
+//               (BN/2)x64 half of the B block per k-block (128-byte swizzle,
+//               no multicast) into a STAGES-deep shared-memory ring, the
+//               completions landing on the leader CTA's barriers;
+//   warp 1      allocates 2*BN TMEM columns in both CTAs; on the leader,
+//               lane 0 issues tcgen05.mma.cta_group::2 (256 x BN x 16 per
+//               instruction) and commits to both CTAs' barriers;
 //   warps 2..   epilogue, in groups of four warps (one per TMEM lane
 //               quadrant): each thread owns one accumulator row and its
 //               group's share of the columns, reads them with tcgen05.ld and
-//               applies a fused epilogue.
+//               applies a fused epilogue; most epilogues turn their rows
+//               around in a per-warp shared-memory scratch so that global
+//               memory is written (and the residual read) in full lines.
 // Two accumulator buffers let the epilogue of tile i overlap the mainloop of
 // tile i+1.  Every mbarrier wait is bounded (see common.cuh).
 #include <cstdio>
