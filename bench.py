@@ -35,6 +35,7 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 
 from synth import workloads as W  # noqa: E402
+from synth.rng import Stream  # noqa: E402
 
 METRIC = "candidate scores/sec on 1 B200 (Qwen3-0.6B shape, K=100) + % of roofline"
 UNIT = "candidate scores/s"
@@ -395,15 +396,47 @@ def run_gather(args, rank: int, world: int, local_rank: int) -> None:
 
 
 LATENCY_CALLS = {1: 200, 8: 100, 64: 40}
+OPEN_LOOP_REQUESTS = 1024
+SEED_OPEN_LOOP = 7007
+
+
+def open_loop_run(rk, packed, arrive_s, cap: int) -> np.ndarray:
+    """Serve requests that arrive at the given times (seconds from start):
+    each call takes every request that has arrived and is not yet served, at
+    most `cap`, scores them through duolm_score and completes them together.
+    Returns each request's latency (completion - arrival) in ms."""
+    n = len(packed)
+    done = np.zeros(n)
+    t0 = time.perf_counter()
+    i = 0
+    while i < n:
+        now = time.perf_counter() - t0
+        if arrive_s[i] > now:
+            time.sleep(arrive_s[i] - now)
+            now = time.perf_counter() - t0
+        j = i
+        while j < n and j - i < cap and arrive_s[j] <= now:
+            j += 1
+        batch = packed[i:j]
+        prefix = np.concatenate([p for p, _, _ in batch]).astype(np.int32)
+        poff = np.concatenate([[0], np.cumsum([len(p) for p, _, _ in batch])]).astype(np.int64)
+        branch = np.concatenate([b for _, b, _ in batch]).astype(np.int32)
+        coff = np.concatenate([[0], np.cumsum([k for _, _, k in batch])]).astype(np.int64)
+        rk.score(prefix, poff, branch, coff, 1)
+        done[i:j] = time.perf_counter() - t0
+        i = j
+    return (done - arrive_s) * 1e3
 
 
 def run_latency(args, rank: int, world: int, local_rank: int) -> None:
-    """Closed-loop latency of the public call: for C in {1, 8, 64}, each call
-    scores a fresh batch of C requests of the 64-request recipe from host
-    buffers (duolm_score: validation, packing, host->device plan copy, the
-    pass, scores back), timed on the host clock around the blocking call;
-    p50/p99 over the calls, with the CUDA graph on and off.  A request's
-    latency is its call's (no queueing: one call at a time)."""
+    """Latency of the public call.  Closed loop: for C in {1, 8, 64}, each
+    call scores a fresh batch of C requests of the 64-request recipe from
+    host buffers (duolm_score: validation, packing, host->device plan copy,
+    the pass, scores back), timed on the host clock around the blocking call;
+    p50/p99 over the calls, with the CUDA graph on and off.  Open loop:
+    requests arrive as a Poisson stream at 50% and 90% of the closed-loop
+    capacity at C, and a server loop scores whatever has arrived (at most C
+    per call); p50/p99 of each request's arrival-to-completion time."""
     import torch
 
     import shared_prefix_item_b200 as S
@@ -412,6 +445,7 @@ def run_latency(args, rank: int, world: int, local_rank: int) -> None:
     rk = S.Ranker(shape, W.model_weights(shape), device=local_rank)
     table_note = load_table(rk, 100_000, shape.d)
     out = {}
+    capacity = {}
     for C, n_calls in LATENCY_CALLS.items():
         batches = [W.c64(n_requests=C, shard=1000 + i).packed() for i in range(n_calls)]
         rk.reserve(max(int(len(b[0]) + len(b[2])) for b in batches), C, C * 100)
@@ -429,7 +463,27 @@ def run_latency(args, rank: int, world: int, local_rank: int) -> None:
             res["graph" if graph else "eager"] = {"p50_ms": float(np.percentile(t, 50)),
                                                   "p99_ms": float(np.percentile(t, 99)),
                                                   "mean_ms": float(t.mean()), "calls": n_calls}
+            if graph:
+                capacity[C] = C / (float(np.median(t)) / 1e3)  # requests/s when every call is full
         out[f"C={C}"] = res
+    # open loop: Poisson arrivals; the server scores whatever has arrived
+    # (at most C requests) each call, one call at a time
+    pool = W.c64(n_requests=OPEN_LOOP_REQUESTS, shard=2000).requests
+    packed = [(r.prefix_ids, r.branch_ids.reshape(-1), r.K) for r in pool]
+    arrivals_u = Stream(SEED_OPEN_LOOP, 0).uniform(OPEN_LOOP_REQUESTS)
+    sizes = sorted((len(p) + len(b) for p, b, _ in packed), reverse=True)
+    rk.reserve(sum(sizes[:64]), 64, 64 * 100)  # any batch fits: no growth (and no re-capture) mid-run
+    open_loop = {}
+    for C in LATENCY_CALLS:
+        for load in (0.5, 0.9):
+            rate = load * capacity[C]
+            gaps = -np.log1p(-arrivals_u) / rate  # exponential inter-arrival times
+            for graph in (True, False):
+                rk.set_graph(graph)
+                lat = open_loop_run(rk, packed, np.cumsum(gaps), C)
+                open_loop[f"C={C} load={load} {'graph' if graph else 'eager'}"] = {
+                    "rate_req_per_s": rate, "p50_ms": float(np.percentile(lat, 50)),
+                    "p99_ms": float(np.percentile(lat, 99)), "requests": len(lat)}
     if rank == 0:
         print(json.dumps({
             "metric": "per-call latency of duolm_score, closed loop (p99, C=64, graph)",
@@ -439,6 +493,7 @@ def run_latency(args, rank: int, world: int, local_rank: int) -> None:
             "config": {"workload": "fresh batches of C requests of the 64-request recipe (K=100, b=1) per call",
                        "table": table_note, "timing": "host clock around the blocking call"},
             "latency": out,
+            "open_loop": open_loop,
         }), flush=True)
     rk.close()
 

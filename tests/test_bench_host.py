@@ -28,3 +28,25 @@ def test_traffic_entries_match_the_current_kernel_sources():
             assert e["dram_bytes_per_launch"] > 0
             got = bench.captured_traffic(kind, cfg)
             assert got is None or got == e["dram_bytes_per_launch"]
+
+
+def test_open_loop_server_serves_every_request_in_arrival_order():
+    import time
+
+    import numpy as np
+
+    class FakeRanker:  # a call takes 2 ms plus 0.1 ms per request
+        def __init__(self):
+            self.batches = []
+
+        def score(self, prefix, poff, branch, coff, b):
+            self.batches.append(len(poff) - 1)
+            time.sleep(0.002 + 0.0001 * (len(poff) - 1))
+
+    n = 60
+    packed = [(np.arange(5, dtype=np.int32), np.arange(3, dtype=np.int32), 3) for _ in range(n)]
+    arrive = np.cumsum(np.full(n, 0.0005))  # faster than the server: batches form
+    rk = FakeRanker()
+    lat = bench.open_loop_run(rk, packed, arrive, cap=8)
+    assert len(lat) == n and np.all(lat > 0)
+    assert sum(rk.batches) == n and max(rk.batches) <= 8 and max(rk.batches) > 1
