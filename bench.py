@@ -28,6 +28,7 @@ import subprocess
 import sys
 import threading
 import time
+from typing import Optional
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
@@ -278,6 +279,32 @@ def oracle_time(wl: W.Workload, requests, warmup: int = 1, independent_cands: in
         per.append(time.perf_counter() - t)
         n += req.K
     return per, n
+
+
+def compile_rate(wl: W.Workload, reps: int = 20) -> Optional[dict]:
+    """Host request compilation (duolm_compile) of the whole batch from its
+    records, on all host threads and on one: requests/s and candidates/s."""
+    import shared_prefix_item_b200 as S
+    if wl.template is None:
+        return None
+    t = wl.template
+    hist, hoff, fb, foff, cand, coff = wl.records()
+    out = {}
+    for label, nt in [("all_threads", 0), ("one_thread", 1)]:
+        def once():
+            return S.compile_requests(wl.model.vocab, t.marker, wl.m, t.instr, t.header,
+                                      t.branch_header[: wl.branch_len - wl.m], hist, hoff, fb, foff, cand, coff,
+                                      wl.n_items // wl.m, nt)
+        once()
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            once()
+        sec = (time.perf_counter() - t0) / reps
+        out[label] = {"us_per_batch": round(sec * 1e6, 1), "requests_per_s": round(len(wl.requests) / sec),
+                      "cand_per_s": round(wl.n_candidates / sec)}
+    out["threads"] = os.cpu_count()
+    out["note"] = "records (item ids, feedback tokens) to packed ids, output arrays included; not in the timed step"
+    return out
 
 
 def cpu_count() -> int:
@@ -638,6 +665,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
             "gpu_launches": launches * args.steps,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
+            "host_compile": compile_rate(wl),
         }
         print(json.dumps(line), flush=True)
     rk.close()

@@ -164,11 +164,58 @@ int64_t duolm_launches_per_execute(const duolm_ctx *ctx);
 
 /* Text of the last failure on this context ("" if none).  Valid until the
  * next call on the context.  With ctx == NULL: the reason the calling
- * thread's last duolm_model_load failed. */
+ * thread's last context-free call (duolm_model_load, duolm_compile) failed. */
 const char *duolm_last_error(const duolm_ctx *ctx);
 
 /* Free every device resource of the context (NULL is ignored). */
 void duolm_destroy(duolm_ctx *ctx);
+
+/* Template text of one ranker prompt format (see duolm_compile). */
+typedef struct {
+  int32_t vocab;                 /* V: the VID of table row i is V + i */
+  int32_t marker;                /* token before each history item's VIDs */
+  int32_t m;                     /* table rows per item (1: one vector per item) */
+  const int32_t *instr;          /* instruction tokens at the start of every prefix */
+  int32_t n_instr;
+  const int32_t *header;         /* tokens after the history, ending the prefix */
+  int32_t n_header;
+  const int32_t *branch_header;  /* tokens before a candidate's VIDs in its branch */
+  int32_t n_branch_header;
+} duolm_template;
+
+/*
+ * duolm_compile -- build the packed layout of duolm_prepare / duolm_score
+ * from request records, on several host threads (DuoLM summary page,
+ * 方法步骤详情 step 3: requests carry item ids and feedback, the runtime
+ * builds the token sequence; the pages name this input compilation as the
+ * host bottleneck at high request rates).  Needs no context and no GPU.
+ * Request r's prefix is
+ *   instr, then for each of its history items h: marker, the VIDs
+ *   V + h m .. V + h m + m - 1, the feedback tokens of h; then header;
+ * its candidates c each get a branch of branch_len = n_branch_header + m
+ * tokens: branch_header, then the VIDs V + c m .. V + c m + m - 1.
+ *   hist_items [hist_offsets[n_requests]] (int64), hist_offsets [n_requests + 1];
+ *   feedback [feedback_offsets[H]] (int32 tokens < V), feedback_offsets
+ *     [H + 1] with H = hist_offsets[n_requests] (one entry per history item);
+ *   cand_items [cand_offsets[n_requests]], cand_offsets [n_requests + 1]
+ *     (every request has at least one candidate);
+ *   n_items: table items (ids must be < n_items); n_threads > 0: that many
+ *     worker threads (at most n_requests), <= 0: one per 256K output tokens,
+ *     at most the host's hardware threads.
+ * Output (caller-owned host arrays): prefix_ids [prefix_capacity] and
+ * prefix_offsets [n_requests + 1]; branch_ids [branch_capacity], candidate
+ * c's branch at c * branch_len (the candidate offsets are cand_offsets).
+ * Returns DUOLM_E_ARG (null pointers, bad template), DUOLM_E_OFFSETS,
+ * DUOLM_E_EMPTY (a request without candidates), DUOLM_E_ID (an item, token
+ * or template id out of range; the outputs are then incomplete),
+ * DUOLM_E_CAPACITY (an output array too small; nothing written but
+ * prefix_offsets).  duolm_last_error(NULL) holds the reason.
+ */
+int duolm_compile(const duolm_template *tpl, int n_requests, const int64_t *hist_items,
+                  const int64_t *hist_offsets, const int32_t *feedback, const int64_t *feedback_offsets,
+                  const int64_t *cand_items, const int64_t *cand_offsets, int64_t n_items, int n_threads,
+                  int32_t *prefix_ids, int64_t prefix_capacity, int64_t *prefix_offsets, int32_t *branch_ids,
+                  int64_t branch_capacity);
 
 /*
  * duolm_gather -- the hot path's first step alone: the virtual-id gather of

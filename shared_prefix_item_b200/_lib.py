@@ -37,6 +37,13 @@ class ModelDesc(ctypes.Structure):
                 ("dtype", ctypes.c_int)]
 
 
+class Template(ctypes.Structure):
+    _fields_ = [("vocab", ctypes.c_int32), ("marker", ctypes.c_int32), ("m", ctypes.c_int32),
+                ("instr", ctypes.c_void_p), ("n_instr", ctypes.c_int32),
+                ("header", ctypes.c_void_p), ("n_header", ctypes.c_int32),
+                ("branch_header", ctypes.c_void_p), ("n_branch_header", ctypes.c_int32)]
+
+
 def _load():
     if not os.path.exists(lib_path):
         raise ImportError(f"{lib_path} is missing: build it with `python -m shared_prefix_item_b200.build`")
@@ -68,6 +75,7 @@ def _load():
         "duolm_debug_wait_timeout": (I, [VP]),
         "duolm_embedding_rho_static": (I, [VP, I, I64, I, VP, VP]),
         "duolm_gather": (I, [VP, VP, I64, VP, VP, VP]),
+        "duolm_compile": (I, [P(Template), I, VP, VP, VP, VP, VP, VP, I64, I, VP, I64, VP, VP, I64]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -89,6 +97,31 @@ def embedding_rho_static(embed_dev: int, dtype: int, vocab: int, d: int, rho_out
                                         ctypes.c_void_p(rho_out_dev), ctypes.c_void_p(stream or 0))
     if rc != 0:
         raise DuolmError(rc, f"duolm_embedding_rho_static(vocab={vocab}, d={d}, dtype={dtype}) failed")
+
+
+def compile_requests(vocab: int, marker: int, m: int, instr, header, branch_header, hist_items, hist_offsets,
+                     feedback, feedback_offsets, cand_items, cand_offsets, n_items: int, n_threads: int = 0):
+    """duolm_compile: request records -> (prefix_ids, prefix_offsets,
+    branch_ids, cand_offsets, branch_len), host arrays in the layout
+    duolm_prepare / duolm_score take."""
+    ins, hdr, bh = (np.ascontiguousarray(x, np.int32) for x in (instr, header, branch_header))
+    tpl = Template(int(vocab), int(marker), int(m), ins.ctypes.data, len(ins), hdr.ctypes.data, len(hdr),
+                   bh.ctypes.data, len(bh))
+    hi, ho = np.ascontiguousarray(hist_items, np.int64), np.ascontiguousarray(hist_offsets, np.int64)
+    fb, fo = np.ascontiguousarray(feedback, np.int32), np.ascontiguousarray(feedback_offsets, np.int64)
+    ci, co = np.ascontiguousarray(cand_items, np.int64), np.ascontiguousarray(cand_offsets, np.int64)
+    R = len(ho) - 1
+    n_hist = np.diff(ho)
+    cap = int(R * (len(ins) + len(hdr)) + n_hist.sum() * (1 + m) + len(fb))
+    b = len(bh) + m
+    prefix = np.empty(max(cap, 1), np.int32)
+    poff = np.empty(R + 1, np.int64)
+    branch = np.empty(max(int(co[-1]) * b, 1), np.int32)
+    rc = lib.duolm_compile(ctypes.byref(tpl), R, _p(hi), _p(ho), _p(fb), _p(fo), _p(ci), _p(co), int(n_items),
+                           int(n_threads), _p(prefix), prefix.size, _p(poff), _p(branch), branch.size)
+    if rc != 0:
+        raise DuolmError(rc, lib.duolm_last_error(None).decode())
+    return prefix[:int(poff[-1])], poff, branch[:int(co[-1]) * b], co, b
 
 
 def _arr(a, dtype) -> np.ndarray:

@@ -22,6 +22,10 @@
 
 using namespace duolm;
 
+// reason of the calling thread's last failed call that has no context
+// (duolm_model_load, duolm_compile); read by duolm_last_error(NULL)
+thread_local std::string g_noctx_err;
+
 namespace {
 
 constexpr int kMaxPos = 32768;   // position ids must stay below this
@@ -103,7 +107,6 @@ struct duolm_ctx {
 
 namespace {
 
-thread_local std::string g_load_err;  // reason of the last failed duolm_model_load
 
 int fail(duolm_ctx* c, int code, const char* fmt, ...) {
   char buf[512];
@@ -472,7 +475,7 @@ int duolm_model_load(const duolm_model_desc* desc, const void* const* host_weigh
   ctx->group = G;
   ctx->rows_per_item = ctx->f16 ? attention_tc_rows_per_item(G) : 64;
   auto bail = [&](int rc) {
-    g_load_err = ctx->err.empty() ? "model_load failed (code " + std::to_string(rc) + ")" : ctx->err;
+    g_noctx_err = ctx->err.empty() ? "model_load failed (code " + std::to_string(rc) + ")" : ctx->err;
     duolm_destroy(ctx);
     return rc;
   };
@@ -914,7 +917,7 @@ int duolm_set_graph(duolm_ctx* ctx, int enabled) {
 
 int64_t duolm_launches_per_execute(const duolm_ctx* ctx) { return ctx ? ctx->launches : 0; }
 
-const char* duolm_last_error(const duolm_ctx* ctx) { return ctx ? ctx->err.c_str() : g_load_err.c_str(); }
+const char* duolm_last_error(const duolm_ctx* ctx) { return ctx ? ctx->err.c_str() : g_noctx_err.c_str(); }
 
 void duolm_destroy(duolm_ctx* ctx) {
   if (!ctx) return;

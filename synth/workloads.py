@@ -117,6 +117,7 @@ class Request:
     branch_ids: np.ndarray          # int32 [K, b] ranker ids; last column is the candidate VID
     history_items: np.ndarray = field(default_factory=lambda: np.zeros(0, np.int64))
     cand_items: np.ndarray = field(default_factory=lambda: np.zeros(0, np.int64))
+    feedback: List[np.ndarray] = field(default_factory=list)  # feedback tokens per history item
 
     @property
     def L(self) -> int:
@@ -135,6 +136,8 @@ class Workload:
     branch_len: int
     requests: List[Request]
     note: str = ""
+    template: Optional["_Template"] = None  # the prompt text the requests were built from
+    m: int = 1                              # table rows per item
 
     @property
     def n_candidates(self) -> int:
@@ -155,6 +158,19 @@ class Workload:
         coff = np.zeros(len(self.requests) + 1, np.int64)
         coff[1:] = np.cumsum([r.K for r in self.requests])
         return prefix, poff, branch, coff
+
+    def records(self):
+        """The requests as records (item ids and feedback tokens, no ids of
+        the ranker's sequence): history items + offsets, feedback tokens +
+        per-history-item offsets, candidate items + offsets."""
+        def flat(arrs, dtype):
+            off = np.zeros(len(arrs) + 1, np.int64)
+            off[1:] = np.cumsum([len(a) for a in arrs])
+            return (np.concatenate(arrs).astype(dtype) if arrs else np.zeros(0, dtype)), off
+        hist, hoff = flat([r.history_items for r in self.requests], np.int64)
+        fb, foff = flat([f for r in self.requests for f in r.feedback], np.int32)
+        cand, coff = flat([r.cand_items for r in self.requests], np.int64)
+        return hist, hoff, fb, foff, cand, coff
 
 
 class _Template:
@@ -205,8 +221,10 @@ def make_request(s: Stream, tpl: _Template, vocab: int, n_items: int, n_hist: in
     hist = item_draw(s, n_hist)
     cands = item_draw(s, n_cand, exclude=hist)
     parts = [tpl.instr]
+    fbs = []
     for i, it in enumerate(hist):
         fb = s.integers(int(feedback_lens[i]), 0, vocab)
+        fbs.append(fb)
         parts += [np.array([tpl.marker, vocab + it]), fb]
     parts.append(tpl.header)
     prefix = np.concatenate([np.asarray(p, np.int64) for p in parts]).astype(np.int32)
@@ -217,7 +235,7 @@ def make_request(s: Stream, tpl: _Template, vocab: int, n_items: int, n_hist: in
         else:
             branch[:, :-1] = np.broadcast_to(tpl.branch_header[: branch_len - 1], (n_cand, branch_len - 1))
     branch[:, -1] = vocab + cands
-    return Request(prefix, branch.astype(np.int32), hist, cands)
+    return Request(prefix, branch.astype(np.int32), hist, cands, fbs)
 
 
 def make_mv_request(s: Stream, tpl: _Template, vocab: int, n_items: int, m: int, n_hist: int, feedback_lens,
@@ -229,13 +247,15 @@ def make_mv_request(s: Stream, tpl: _Template, vocab: int, n_items: int, m: int,
     hist = s.distinct(n_hist, 0, n_items)
     cands = s.distinct(n_cand, 0, n_items, hist)
     parts = [tpl.instr]
+    fbs = []
     for i, it in enumerate(hist):
         fb = s.integers(int(feedback_lens[i]), 0, vocab)
+        fbs.append(fb)
         parts += [np.array([tpl.marker]), vocab + it * m + np.arange(m), fb]
     parts.append(tpl.header)
     prefix = np.concatenate([np.asarray(p, np.int64) for p in parts]).astype(np.int32)
     branch = vocab + cands[:, None] * m + np.arange(m)[None, :]
-    return Request(prefix, branch.astype(np.int32), hist, cands)
+    return Request(prefix, branch.astype(np.int32), hist, cands, fbs)
 
 
 def fir(m: int = 8, n_requests: int = 64, shard: int = 0) -> Workload:
@@ -251,7 +271,7 @@ def fir(m: int = 8, n_requests: int = 64, shard: int = 0) -> Workload:
         h = int(s.integers(1, 1, 21)[0])
         f = s.integers(h, 8, 49)
         reqs.append(make_mv_request(s, tpl, model.vocab, n_items, m, h, f, 100))
-    return Workload(f"fir-m{m}", model, n_items * m, m, reqs)
+    return Workload(f"fir-m{m}", model, n_items * m, m, reqs, template=tpl, m=m)
 
 
 def custom_fir(model: ModelShape, n_items: int, seed: int, n_requests: int, n_hist: int, feedback: int,
@@ -262,7 +282,7 @@ def custom_fir(model: ModelShape, n_items: int, seed: int, n_requests: int, n_hi
     tpl = _Template(s, model.vocab, 3, 2, 0)
     reqs = [make_mv_request(s, tpl, model.vocab, n_items, m, n_hist, [feedback] * n_hist, n_cand)
             for _ in range(n_requests)]
-    return Workload(f"custom-fir-m{m}", model, n_items * m, m, reqs)
+    return Workload(f"custom-fir-m{m}", model, n_items * m, m, reqs, template=tpl, m=m)
 
 
 def tiny(seed_offset: int = 0) -> Workload:
@@ -271,7 +291,7 @@ def tiny(seed_offset: int = 0) -> Workload:
     s = Stream(SEED_REQUESTS + 0 + seed_offset, 0)
     tpl = _Template(s, m.vocab, 8, 0, 0)
     r = make_request(s, tpl, m.vocab, 64, 4, [8] * 4, 8, 1)
-    return Workload("tiny", m, 64, 1, [r])
+    return Workload("tiny", m, 64, 1, [r], template=tpl)
 
 
 def c1(shard: int = 0) -> Workload:
@@ -280,7 +300,7 @@ def c1(shard: int = 0) -> Workload:
     s = Stream(SEED_REQUESTS + 1, shard)
     tpl = _Template(s, m.vocab, 32, 4, 0)
     r = make_request(s, tpl, m.vocab, 100_000, 10, [24] * 10, 100, 1)
-    return Workload("c1", m, 100_000, 1, [r])
+    return Workload("c1", m, 100_000, 1, [r], template=tpl)
 
 
 def c64(n_requests: int = 64, shard: int = 0) -> Workload:
@@ -295,7 +315,7 @@ def c64(n_requests: int = 64, shard: int = 0) -> Workload:
         h = int(s.integers(1, 1, 21)[0])
         f = s.integers(h, 8, 49)
         reqs.append(make_request(s, tpl, m.vocab, 100_000, h, f, 100, 1))
-    return Workload("c64", m, 100_000, 1, reqs)
+    return Workload("c64", m, 100_000, 1, reqs, template=tpl)
 
 
 def stress(n_requests: int = 16, shard: int = 0) -> Workload:
@@ -305,7 +325,7 @@ def stress(n_requests: int = 16, shard: int = 0) -> Workload:
     s = Stream(SEED_REQUESTS + 3, shard)
     tpl = _Template(s, m.vocab, 32, 0, 3)
     reqs = [make_request(s, tpl, m.vocab, 100_000, 50, [40] * 50, 256, 4) for _ in range(n_requests)]
-    return Workload("stress", m, 100_000, 4, reqs)
+    return Workload("stress", m, 100_000, 4, reqs, template=tpl)
 
 
 def catalog(concurrency: int, shard: int = 0) -> Workload:
@@ -318,7 +338,7 @@ def catalog(concurrency: int, shard: int = 0) -> Workload:
     draw = _zipf_sampler(n_items, 1.1)
     reqs = [make_request(s, tpl, m.vocab, n_items, 10, [24] * 10, 100, 1, item_draw=draw)
             for _ in range(concurrency)]
-    return Workload(f"catalog-c{concurrency}", m, n_items, 1, reqs)
+    return Workload(f"catalog-c{concurrency}", m, n_items, 1, reqs, template=tpl)
 
 
 def custom(model: ModelShape, n_items: int, seed: int, n_requests: int, n_hist, feedback,
@@ -341,7 +361,8 @@ def custom(model: ModelShape, n_items: int, seed: int, n_requests: int, n_hist, 
         k = pick(n_cand)
         reqs.append(make_request(s, tpl, model.vocab, n_items, h, f, k, branch_len,
                                  random_branch_header=random_branch_header))
-    return Workload(f"custom-{seed}", model, n_items, branch_len, reqs)
+    return Workload(f"custom-{seed}", model, n_items, branch_len, reqs,
+                    template=None if random_branch_header else tpl)
 
 
 CONFIGS = {"tiny": tiny, "c1": c1, "c64": c64, "stress": stress}
