@@ -2,7 +2,8 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--config c64|c1|stress|catalog-c64|catalog-c8|catalog-c1]
-                    [--mode mis|independent] [--no-graph] [--skip-cpu] [--profile-steps N]
+                    [--mode mis|independent] [--reuse append|rescore] [--no-graph] [--skip-cpu]
+                    [--profile-steps N]
 
 One step is one pass of the whole hot path (virtual-id gather, 28 decoder
 layers with shared-prefix tree-masked attention, score head) over one batch
@@ -17,6 +18,12 @@ Prints one JSON line (rank 0).  `value` times device-resident batches
 host buffers (validation, packing, host->device copy, pass, scores back).
 `--impl reference` times the oracle (plain fp64 CPU code) on the host cores
 instead, one request of the same workload per step.
+
+`--reuse` runs the same requests from a prefix KV store: `append` stores each
+request's prefix up to its last history item beforehand, and every step
+appends that item and the header (the new history arrives) before scoring;
+`rescore` stores the whole prefix and every step scores the K candidates
+only.  The scores are those of the full sequences either way.
 """
 from __future__ import annotations
 
@@ -97,24 +104,56 @@ def gemm_flops(shape: W.ModelShape, T: int) -> float:
     return 2.0 * T * (d * (qd + 2 * kd) + qd * d + d * 2 * F + F * d) * shape.n_layers
 
 
-def attention_pairs(wl: W.Workload, independent: bool) -> int:
+def attention_pairs(wl: W.Workload, independent: bool, cached=None) -> int:
+    """(query, key) pairs of one pass; with cached[q] prefix tokens of request
+    q already stored, only the queries after them are computed."""
     b = wl.branch_len
     tot = 0
-    for r in wl.requests:
+    for q, r in enumerate(wl.requests):
         L, K = r.L, r.K
+        c = cached[q] if cached is not None else 0
         if independent:
             tot += K * (L + b) * (L + b + 1) // 2
         else:
-            tot += L * (L + 1) // 2 + K * sum(L + i + 1 for i in range(b))
+            tot += (L * (L + 1) - c * (c + 1)) // 2 + K * sum(L + i + 1 for i in range(b))
     return tot
 
 
-def attention_flops(shape: W.ModelShape, wl: W.Workload, independent: bool) -> float:
+def attention_flops(shape: W.ModelShape, wl: W.Workload, independent: bool, cached=None) -> float:
     # QK^T and PV: 2 * head_dim each per (query, key) pair and query head
-    return 4.0 * shape.head_dim * shape.n_q_heads * attention_pairs(wl, independent) * shape.n_layers
+    return 4.0 * shape.head_dim * shape.n_q_heads * attention_pairs(wl, independent, cached) * shape.n_layers
 
 
-def class_flops(shape: W.ModelShape, wl: W.Workload, T: int, independent: bool) -> dict:
+class Reuse:
+    """Arguments of the prefix-reuse runs: `warm` fills the store (request q
+    in slot q), `step` is the batch every timed step runs."""
+
+    def __init__(self, wl: W.Workload, kind: str):
+        R = len(wl.requests)
+        n_header = len(wl.template.header)
+        p, po, b, co = wl.packed()
+        if kind == "append":
+            # everything before the last history item
+            self.cached = [wl.history_offsets(q)[-1] for q in range(R)]
+            keep = [r.L - c - n_header for r, c in zip(wl.requests, self.cached)]
+        elif kind == "rescore":
+            self.cached = [r.L for r in wl.requests]
+            keep = [0] * R
+        else:
+            raise SystemExit(f"unknown --reuse {kind}")
+        warm_ids = np.concatenate([r.prefix_ids[:c] for r, c in zip(wl.requests, self.cached)])
+        warm_off = np.cumsum([0] + self.cached)
+        new_ids = np.concatenate([r.prefix_ids[c:] for r, c in zip(wl.requests, self.cached)])
+        new_off = np.cumsum([0] + [r.L - c for r, c in zip(wl.requests, self.cached)])
+        slots = np.arange(R)
+        self.slot_tokens = max(r.L for r in wl.requests)
+        self.warm = (warm_ids, warm_off, b, co, wl.branch_len, slots, np.zeros(R), self.cached)
+        self.step = (new_ids, new_off, b, co, wl.branch_len, slots, self.cached, keep)
+        self.note = (f"{kind}: {sum(self.cached)} of {sum(r.L for r in wl.requests)} prefix tokens read from "
+                     f"the KV store, {int(new_off[-1])} new prefix tokens per step")
+
+
+def class_flops(shape: W.ModelShape, wl: W.Workload, T: int, independent: bool, cached=None) -> dict:
     """Algorithmic FLOPs per step of each kernel class (multiply-add = 2)."""
     d, qd, kd, F, L = shape.d, shape.q_dim, shape.kv_dim, shape.ffn, shape.n_layers
     return {
@@ -122,7 +161,7 @@ def class_flops(shape: W.ModelShape, wl: W.Workload, T: int, independent: bool) 
         "gemm_o": 2.0 * T * qd * d * L,
         "gemm_gate_up": 2.0 * T * d * 2 * F * L,
         "gemm_down": 2.0 * T * F * d * L,
-        "attention": attention_flops(shape, wl, independent),
+        "attention": attention_flops(shape, wl, independent, cached),
     }
 
 
@@ -548,7 +587,26 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     table_note = load_table(rk, wl.n_items, shape.d)
     rk.set_graph(not args.no_graph)
     p, po, b, co = wl.packed()
-    rk.prepare(p, po, b, co, wl.branch_len, mode)
+    reuse = None
+    if args.reuse:
+        if mode != S.MODE_MIS:
+            raise SystemExit("--reuse needs --mode mis")
+        reuse = Reuse(wl, args.reuse)
+        rk.kv_store_reserve(len(wl.requests), reuse.slot_tokens)
+        rk.score_cached(*reuse.warm)
+
+        def prepare():
+            rk.prepare_cached(*reuse.step)
+
+        def score_host(out):
+            rk.score_cached(*reuse.step, out=out)
+    else:
+        def prepare():
+            rk.prepare(p, po, b, co, wl.branch_len, mode)
+
+        def score_host(out):
+            rk.score(p, po, b, co, wl.branch_len, mode, out=out)
+    prepare()
     n_cand = wl.n_candidates
     T = int(rk.debug_layout()[0].shape[0])
 
@@ -588,12 +646,12 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
 
     # e2e: the public call from host buffers, scores back to the host every step
     out = np.empty(n_cand, np.float32)
-    rk.score(p, po, b, co, wl.branch_len, mode, out=out)
+    score_host(out)
     h2d = rk.plan_bytes()
     barrier()
     start.record(stream)
     for _ in range(args.steps):
-        rk.score(p, po, b, co, wl.branch_len, mode, out=out)
+        score_host(out)
     end.record(stream)
     barrier()
     e2e_ms = start.elapsed_time(end) / args.steps
@@ -601,12 +659,12 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     e2e_value = n_total / (e2e_max / 1e3)
 
     # per-kernel-class device time (eager launches with an event after each)
-    rk.prepare(p, po, b, co, wl.branch_len, mode)
+    prepare()
     prof = rk.profile(max(2, min(args.steps, 5)))
     steps_prof = max(2, min(args.steps, 5))
     pk = peaks()
     indep = mode == S.MODE_INDEPENDENT
-    cf = class_flops(shape, wl, T, indep)
+    cf = class_flops(shape, wl, T, indep, reuse.cached if reuse else None)
     gf = sum(v for k, v in cf.items() if k != "attention")
     af = cf["attention"]
     kernels = {k: {"ms_per_step": round(v[0] / steps_prof, 4), "launches_per_step": v[1] // steps_prof}
@@ -615,6 +673,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     for v in kernels.values():
         v["share"] = round(v["ms_per_step"] / tot_ms, 4) if tot_ms else None
     names = {"gemm_qkv": "gemm_tc_kernel<EpiQkv> (QKV projection, QK-norm, RoPE)",
+             "kv_append": "kv_append_kernel (new prefix K/V into the store)",
              "gemm_o": "gemm_tc_kernel<EpiResid> (O projection + residual)",
              "gemm_gate_up": "gemm_tc_kernel<EpiSwiglu> (gate/up projection + SwiGLU)",
              "gemm_down": "gemm_tc_kernel<EpiResid> (down projection + residual)",
@@ -629,16 +688,18 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
              "unit": "TFLOP/s", "kernel": names[k], "launches_per_step": n_k, "flops_per_launch": fl / n_k,
              "us_per_launch": ms_k * 1e3 / n_k,
              "peak_note": f"{pk['src']} sustained bf16 dense (fp16 runs at the bf16 rate)",
-             "traffic": captured_traffic(k, args.config)}
+             "traffic": None if reuse else captured_traffic(k, args.config)}
         r["frac"] = r["achieved"] / r["peak"]
         if k == "attention":
             r["hbm_gbs_algorithmic"] = attention_bytes(shape, T) / (ms_k / 1e3) / 1e9
+            if reuse:
+                r["note"] = "K/V read from the store not counted in the algorithmic bytes"
         roofs[k] = r
     dom_key = max(roofs, key=lambda k: prof[k][0])
     dominant = roofs[dom_key]
     step_roof_ms = max((gf + af) / (pk["tc_sustained"] * 1e12), 0.0) * 1e3
     cpu = None
-    if rank == 0 and world == 1 and not args.skip_cpu:
+    if rank == 0 and world == 1 and not args.skip_cpu and not reuse:
         per, nc = oracle_time(wl, [0])
         per_i, nc_i = oracle_time(wl, [0], independent_cands=4)
         cpu = {"value": nc / sum(per), "unit": UNIT, "cores": cpu_count(), "kind": "oracle",
@@ -652,9 +713,10 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": (value / PAGES_CAND_PER_S[(args.config, args.mode)]
-                            if (args.config, args.mode) in PAGES_CAND_PER_S else None),
+                            if (args.config, args.mode) in PAGES_CAND_PER_S and not reuse else None),
             "dtype": "f16", "data": "synthetic",
-            "config": {**describe(wl, args.mode, not args.no_graph, world), "table": table_note},
+            "config": {**describe(wl, args.mode, not args.no_graph, world), "table": table_note,
+                       **({"reuse": reuse.note, "tokens_per_step": T} if reuse else {})},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4 * n_cand},
             "roofline": dominant,
             "roofline_step": {"flops_per_step": gf + af, "ms_at_peak": step_roof_ms,
@@ -682,6 +744,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="c64")
     ap.add_argument("--mode", choices=["mis", "independent"], default="mis")
+    ap.add_argument("--reuse", choices=["append", "rescore"], default=None,
+                    help="score from a prefix KV store (see the module docstring)")
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--profile-steps", type=int, default=0,

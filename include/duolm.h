@@ -134,6 +134,59 @@ int duolm_prepare(duolm_ctx *ctx, int n_requests, const int32_t *prefix_ids,
                   const int64_t *cand_offsets, int branch_len, int mode);
 
 /*
+ * Prefix KV reuse (incremental history append; DuoLM summary page, 未来方向
+ * (3): when new history items arrive only their vectors and K/V are added).
+ * A causal prefix's K/V at every layer depend only on the tokens before
+ * them, so a request can start from the K/V an earlier call computed for
+ * the first c tokens of its prefix and run only the tokens after them; its
+ * scores are those of the whole sequence.
+ *
+ * duolm_kv_store_reserve: allocate the store, n_slots slots of slot_tokens
+ * token rows (K and V of every layer and KV head; 2 * n_layers * n_kv_heads
+ * * head_dim * element size bytes per row: 112 KB for the Qwen3-0.6B
+ * shape in fp16).  Frees any previous store and its contents (every slot
+ * length back to 0), drops the prepared batch and the CUDA graph;
+ * n_slots = 0 frees the store.  Synchronous.  DUOLM_E_ARG for negative
+ * sizes or slot_tokens above the position limit (32,768), DUOLM_E_CAPACITY
+ * above 2^31 rows per layer, DUOLM_E_CUDA when the memory is not there.
+ */
+int duolm_kv_store_reserve(duolm_ctx *ctx, int n_slots, int slot_tokens);
+
+/* Tokens whose K/V slot `slot` holds (DUOLM_E_ARG for a bad slot). */
+int duolm_kv_slot_length(const duolm_ctx *ctx, int slot);
+
+/*
+ * duolm_prepare in multi-item mode with per-request prefix reuse.  For
+ * request q (host arrays of n_requests entries):
+ *   slot[q] = -1: as in duolm_prepare (cached[q] and keep[q] must be 0);
+ *   slot[q] = s >= 0: the first cached[q] tokens of the request's prefix
+ *     are the first cached[q] tokens slot s holds (cached[q] <= the slot's
+ *     length); prefix_ids holds only the L_q tokens after them (L_q may be 0
+ *     when cached[q] > 0: new candidates for an unchanged prefix), at
+ *     positions cached[q] .. cached[q] + L_q - 1, and the branches sit at
+ *     position cached[q] + L_q.  The first keep[q] (0 <= keep[q] <= L_q) of
+ *     the new tokens are appended to the slot: once the batch has run, the
+ *     slot holds cached[q] + keep[q] tokens (keep[q] = 0 leaves it as it
+ *     is).  A trailing header is usually left out of keep so that the next
+ *     call can append history before it.
+ * A slot that a request of the batch appends to may not be used by any
+ * other request of the same batch.  Errors as duolm_prepare, plus
+ * DUOLM_E_STATE (no store reserved, or cached[q] above the slot's length),
+ * DUOLM_E_ARG (bad slot, cached, keep or sharing), DUOLM_E_CAPACITY
+ * (cached[q] + keep[q] above slot_tokens).
+ */
+int duolm_prepare_cached(duolm_ctx *ctx, int n_requests, const int32_t *prefix_ids,
+                         const int64_t *prefix_offsets, const int32_t *branch_ids,
+                         const int64_t *cand_offsets, int branch_len, const int32_t *slot,
+                         const int32_t *cached, const int32_t *keep);
+
+/* duolm_prepare_cached + duolm_execute + scores to the host + duolm_sync. */
+int duolm_score_cached(duolm_ctx *ctx, int n_requests, const int32_t *prefix_ids,
+                       const int64_t *prefix_offsets, const int32_t *branch_ids,
+                       const int64_t *cand_offsets, int branch_len, const int32_t *slot,
+                       const int32_t *cached, const int32_t *keep, float *scores_out);
+
+/*
  * Run the ranker on the prepared batch, asynchronously on the context
  * stream.  Scores (fp32, one per candidate, input order) land in the device
  * buffer returned by duolm_scores_device.  Uses the CUDA graph unless
@@ -327,7 +380,8 @@ int duolm_debug_wait_timeout(duolm_ctx *ctx);
 #define DUOLM_PROF_GEMM_GATE_UP 5
 #define DUOLM_PROF_GEMM_DOWN 6
 #define DUOLM_PROF_HEAD 7
-#define DUOLM_PROF_N 8
+#define DUOLM_PROF_KV_APPEND 8
+#define DUOLM_PROF_N 9
 
 /*
  * Run the prepared batch n_steps times kernel by kernel with a CUDA event

@@ -76,6 +76,10 @@ def _load():
         "duolm_embedding_rho_static": (I, [VP, I, I64, I, VP, VP]),
         "duolm_gather": (I, [VP, VP, I64, VP, VP, VP]),
         "duolm_compile": (I, [P(Template), I, VP, VP, VP, VP, VP, VP, I64, I, VP, I64, VP, VP, I64]),
+        "duolm_kv_store_reserve": (I, [VP, I, I]),
+        "duolm_kv_slot_length": (I, [VP, I]),
+        "duolm_prepare_cached": (I, [VP, I, VP, VP, VP, VP, I, VP, VP, VP]),
+        "duolm_score_cached": (I, [VP, I, VP, VP, VP, VP, I, VP, VP, VP, VP]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -225,6 +229,41 @@ class Ranker:
         p, po, b, co = wl.packed()
         return self.score(p, po, b, co, wl.branch_len, mode)
 
+    # ---- prefix KV reuse
+    def kv_store_reserve(self, n_slots: int, slot_tokens: int):
+        self._check(lib.duolm_kv_store_reserve(self.ctx, int(n_slots), int(slot_tokens)))
+
+    def kv_slot_length(self, slot: int) -> int:
+        n = lib.duolm_kv_slot_length(self.ctx, int(slot))
+        if n < 0:
+            raise DuolmError(n, f"kv_slot_length({slot})")
+        return n
+
+    def _cached_args(self, prefix_ids, prefix_offsets, branch_ids, cand_offsets, slot, cached, keep):
+        a = [_arr(prefix_ids, np.int32), _arr(prefix_offsets, np.int64), _arr(branch_ids, np.int32),
+             _arr(cand_offsets, np.int64)]
+        R = a[1].shape[0] - 1
+        s = [_arr(np.broadcast_to(v, (R,)), np.int32) for v in (slot, cached, keep)]
+        return a, s, R
+
+    def prepare_cached(self, prefix_ids, prefix_offsets, branch_ids, cand_offsets, branch_len: int, slot, cached,
+                       keep):
+        """duolm_prepare_cached: request q continues the first cached[q]
+        tokens slot[q] holds and appends keep[q] of its new prefix tokens."""
+        a, s, R = self._cached_args(prefix_ids, prefix_offsets, branch_ids, cand_offsets, slot, cached, keep)
+        self._check(lib.duolm_prepare_cached(self.ctx, R, _p(a[0]), _p(a[1]), _p(a[2]), _p(a[3]), int(branch_len),
+                                             _p(s[0]), _p(s[1]), _p(s[2])))
+        self.n_cand = int(a[3][-1])
+
+    def score_cached(self, prefix_ids, prefix_offsets, branch_ids, cand_offsets, branch_len: int, slot, cached,
+                     keep, out: Optional[np.ndarray] = None) -> np.ndarray:
+        a, s, R = self._cached_args(prefix_ids, prefix_offsets, branch_ids, cand_offsets, slot, cached, keep)
+        if out is None:
+            out = np.empty(int(a[3][-1]), np.float32)
+        self._check(lib.duolm_score_cached(self.ctx, R, _p(a[0]), _p(a[1]), _p(a[2]), _p(a[3]), int(branch_len),
+                                           _p(s[0]), _p(s[1]), _p(s[2]), _p(out)))
+        return out
+
     def set_graph(self, enabled: bool):
         self._check(lib.duolm_set_graph(self.ctx, 1 if enabled else 0))
 
@@ -259,7 +298,8 @@ class Ranker:
     def plan_bytes(self) -> int:
         return int(lib.duolm_plan_bytes(self.ctx))
 
-    PROFILE_CLASSES = ("embed", "gemm_qkv", "attention", "gemm_o", "rmsnorm", "gemm_gate_up", "gemm_down", "head")
+    PROFILE_CLASSES = ("embed", "gemm_qkv", "attention", "gemm_o", "rmsnorm", "gemm_gate_up", "gemm_down", "head",
+                       "kv_append")
 
     def profile(self, n_steps: int) -> dict:
         """Per kernel class: (summed device ms over n_steps, launches)."""

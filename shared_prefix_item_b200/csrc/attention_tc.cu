@@ -10,7 +10,16 @@
 //   kind 0  prefix tokens [row0, row0 + 2R): causal over the prefix;
 //   kind 1  branch tokens (whole candidates): every prefix key tile, then the
 //           tiles of the item's own branch rows under the tree rule.
-// B is left out when the item's rows all fit in A.  One CTA per SM, 384
+// B is left out when the item's rows all fit in A.
+// A request may continue a cached prefix (incremental history append): its
+// first c prefix tokens were computed by an earlier call and their K/V sit
+// in a slot of the per-layer KV store; the batch holds only the tokens after
+// them.  Request-local indices still count from the first cached token, so
+// masks and positions are those of the whole sequence: key tiles
+// [0, ceil(c / 128)) come from the store (keys >= c masked), the remaining
+// prefix tiles start at c and come from this batch's K/V, and query rows
+// start at c.  With c = 0 the item is exactly the uncached one.
+// One CTA per SM, 384
 // threads in three warpgroups:
 //   warps 0-3 softmax of A, warps 4-7 softmax of B: one thread per slot row
 //             (TMEM lane) and 128 keys: load S, mask, row max, P = 2^(s - m)
@@ -68,18 +77,25 @@ enum { B_QFULL0, B_QFULL1, B_QEMPTY0, B_QEMPTY1, B_KFULL0, B_KFULL1, B_VFULL0, B
        B_VEMPTY0, B_VEMPTY1, B_SFULL0, B_SFULL1, B_PFULL0, B_PFULL1, B_OFULL0, B_OFULL1, B_DRAIN, B_COUNT };
 
 struct Item {
-  int tok0, L, K, kvh, branch, row0, q0, nrows, n_prefix_tiles, n_tiles, has_b;
+  // qbase: batch row of request-local index 0 (the first cached token's
+  // index; batch rows hold only indices >= c); slot0: the request's first
+  // store row; tiles [0, n_cached_tiles) are store tiles
+  int qbase, c, slot0, L, K, kvh, branch, row0, q0, nrows, n_cached_tiles, n_prefix_tiles, n_tiles, has_b;
   __device__ int tile_start(int t) const {
-    return t < n_prefix_tiles ? t * kKeys : q0 + (t - n_prefix_tiles) * kKeys;
+    return t < n_cached_tiles ? t * kKeys
+                              : (t < n_prefix_tiles ? c + (t - n_cached_tiles) * kKeys
+                                                    : q0 + (t - n_prefix_tiles) * kKeys);
   }
 };
 
 template <int G>
-__device__ __forceinline__ Item make_item(int4 item, int4 rq, int b) {
+__device__ __forceinline__ Item make_item(int4 item, int4 rq, int2 rx, int b) {
   constexpr int R = kSub / G;  // tokens per sub-tile
   constexpr int R2 = 2 * R;    // tokens per item
   Item m;
-  m.tok0 = rq.x;
+  m.c = rx.x;
+  m.slot0 = rx.y;
+  m.qbase = rq.x - rx.x;
   m.L = rq.y;
   m.K = rq.z;
   m.kvh = item.y;
@@ -88,7 +104,8 @@ __device__ __forceinline__ Item make_item(int4 item, int4 rq, int b) {
   m.q0 = m.branch ? m.L + m.row0 : m.row0;
   m.nrows = m.branch ? min((R2 / b) * b, m.K * b - m.row0) : min(R2, m.L - m.row0);
   const int kend = m.branch ? m.L : min(m.row0 + R2, m.L);
-  m.n_prefix_tiles = (kend + kKeys - 1) / kKeys;
+  m.n_cached_tiles = (m.c + kKeys - 1) / kKeys;
+  m.n_prefix_tiles = m.n_cached_tiles + (kend - m.c + kKeys - 1) / kKeys;
   m.n_tiles = m.n_prefix_tiles + (m.branch ? (m.nrows + kKeys - 1) / kKeys : 0);
   m.has_b = m.nrows > R;
   return m;
@@ -103,11 +120,14 @@ template <int G>
 struct ItemStream {
   const int4* items;
   const int4* reqs;
+  const int2* reqx;
   int n, step, b;
   int it;
   int4 d1, d2, r1;  // descriptor of it + step, it + 2 step; request of it + step
-  __device__ ItemStream(const PlanHdr* plan, int cta, int n_ctas, int b_)
-      : items(plan_array<int4>(plan, plan->off_items)), reqs(plan_array<int4>(plan, plan->off_req)), b(b_) {
+  int2 x1;          // cached prefix of that request
+  __device__ ItemStream(const PlanHdr* plan, const int2* reqx_, int cta, int n_ctas, int b_)
+      : items(plan_array<int4>(plan, plan->off_items)), reqs(plan_array<int4>(plan, plan->off_req)), reqx(reqx_),
+        b(b_) {
     if (plan->att_ctas == n_ctas) {
       const int32_t* off = plan_array<int32_t>(plan, plan->off_cta);
       it = off[cta];
@@ -122,15 +142,17 @@ struct ItemStream {
     d1 = it < n ? items[it] : z;
     d2 = it + step < n ? items[it + step] : z;
     r1 = reqs[d1.x];
+    x1 = reqx[d1.x];
   }
   __device__ bool valid() const { return it < n; }
   // the current item; advances the prefetch window
   __device__ Item next() {
-    const Item m = make_item<G>(d1, r1, b);
+    const Item m = make_item<G>(d1, r1, x1, b);
     const int4 z = make_int4(0, 0, 0, 0);
     it += step;
     d1 = d2;
     r1 = reqs[d1.x];
+    x1 = reqx[d1.x];
     d2 = it + step < n ? items[it + step] : z;
     return m;
   }
@@ -141,8 +163,10 @@ struct ItemStream {
 template <int G>
 __global__ void __launch_bounds__(kThreads, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                        const __grid_constant__ CUtensorMap tmV, const PlanHdr* __restrict__ plan, int64_t kv_rows,
-                        int n_q_heads, float scale_log2, __half* __restrict__ o, DevStatus* st) {
+                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKs,
+                        const __grid_constant__ CUtensorMap tmVs, const PlanHdr* __restrict__ plan,
+                        const int2* __restrict__ reqx, int64_t kv_rows, int64_t store_rows, int n_q_heads,
+                        float scale_log2, __half* __restrict__ o, DevStatus* st) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -159,6 +183,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&tmQ);
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
+    prefetch_tensormap(&tmKs);
+    prefetch_tensormap(&tmVs);
     for (int i = 0; i < B_COUNT; ++i)
       mbar_init(bar(i), (i == B_PFULL0 || i == B_PFULL1) ? (uint32_t)kSoftmaxWG : 1u);
     fence_barrier_init();
@@ -185,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tmem + lane_off + 128 * X, tO = tmem + lane_off + 256 + 128 * X;
     uint32_t n_xt = 0, n_xi = 0;
     bool ok = true;
-    for (ItemStream<G> is(plan, blockIdx.x, gridDim.x, b); is.valid() && ok;) {
+    for (ItemStream<G> is(plan, reqx, blockIdx.x, gridDim.x, b); is.valid() && ok;) {
       const Item m = is.next();
       if (X == 1 && !m.has_b) continue;
       const int rl = X * R + r / G;  // row of the item (token offset from q0)
@@ -207,13 +233,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 32; ++j) tmem_ld_fence(sr[c][j]);
         const int k0 = m.tile_start(t);
         const bool is_branch_tile = t >= m.n_prefix_tiles;
-        const bool need_mask = is_branch_tile || (!m.branch && k0 + kKeys > m.row0) || (m.branch && k0 + kKeys > m.L);
+        const bool is_cached_tile = t < m.n_cached_tiles;
+        const bool need_mask = is_branch_tile || (is_cached_tile && k0 + kKeys > m.c) ||
+                               (!is_cached_tile && ((!m.branch && k0 + kKeys > m.row0) || (m.branch && k0 + kKeys > m.L)));
         if (need_mask) {
           // this row's visible keys in the tile are one window [lo0, lo0 + n)
           // of tile-local indices: its own branch keys in a branch tile, the
+          // cached keys (all below every query row) in a store tile, the
           // prefix keys up to pre_hi otherwise
           const int lo = is_branch_tile ? kr.br_lo - k0 : 0;
-          const int hi = is_branch_tile ? kr.br_hi - k0 : kr.pre_hi - k0;  // inclusive
+          const int hi = (is_branch_tile ? kr.br_hi : (is_cached_tile ? m.c - 1 : kr.pre_hi)) - k0;  // inclusive
           const uint32_t lo0 = (uint32_t)max(lo, 0);
           const uint32_t n = (uint32_t)max(0, min(hi, kKeys - 1) - max(lo, 0) + 1);
 #pragma unroll
@@ -279,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++n_xi;
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const bool valid = rl < m.nrows;
-      __half* dst = o + (((int64_t)m.tok0 + m.q0 + rl) * n_q_heads + m.kvh * G + (r % G)) * kHD;
+      __half* dst = o + (((int64_t)m.qbase + m.q0 + rl) * n_q_heads + m.kvh * G + (r % G)) * kHD;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         float v[32];
@@ -302,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         uint32_t n_kv = 0, n_xi[2] = {0, 0};
         bool ok = true;
-        for (ItemStream<G> is(plan, blockIdx.x, gridDim.x, b); is.valid() && ok;) {
+        for (ItemStream<G> is(plan, reqx, blockIdx.x, gridDim.x, b); is.valid() && ok;) {
           const Item m = is.next();
 #pragma unroll
           for (int X = 0; X < 2; ++X) {
@@ -314,26 +343,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(bar(B_QFULL0 + X), 2 * kHalf);
             for (int h = 0; h < 2; ++h)
               tma_load_3d(&tmQ, sbase + kQOff + (2 * X + h) * kHalf, bar(B_QFULL0 + X), h * 64, m.kvh * G,
-                          m.tok0 + m.q0 + X * R);
+                          m.qbase + m.q0 + X * R);
             ++n_xi[X];
           }
           for (int t = 0; t < m.n_tiles && ok; ++t, ++n_kv) {
             const uint32_t slot = n_kv & 1, use = n_kv >> 1;
-            const int y = (int)((int64_t)m.kvh * kv_rows + m.tok0 + m.tile_start(t));
+            // a store tile reads the request's slot, every other tile this batch's K/V
+            const bool cached = t < m.n_cached_tiles;
+            const CUtensorMap* mk = cached ? &tmKs : &tmK;
+            const CUtensorMap* mv = cached ? &tmVs : &tmV;
+            const int y = cached ? (int)((int64_t)m.kvh * store_rows + m.slot0 + m.tile_start(t))
+                                 : (int)((int64_t)m.kvh * kv_rows + m.qbase + m.tile_start(t));
             if (!mbar_wait(bar(B_KEMPTY0 + slot), (use & 1u) ^ 1u, st, 41)) {
               ok = false;
               break;
             }
             mbar_arrive_expect_tx(bar(B_KFULL0 + slot), 2 * kHalf);
             for (int h = 0; h < 2; ++h)
-              tma_load_2d(&tmK, sbase + kKOff + (2 * slot + h) * kHalf, bar(B_KFULL0 + slot), h * 64, y);
+              tma_load_2d(mk, sbase + kKOff + (2 * slot + h) * kHalf, bar(B_KFULL0 + slot), h * 64, y);
             if (!mbar_wait(bar(B_VEMPTY0 + slot), (use & 1u) ^ 1u, st, 42)) {
               ok = false;
               break;
             }
             mbar_arrive_expect_tx(bar(B_VFULL0 + slot), 2 * kHalf);
             for (int h = 0; h < 2; ++h)
-              tma_load_2d(&tmV, sbase + kVOff + (2 * slot + h) * kHalf, bar(B_VFULL0 + slot), h * 64, y);
+              tma_load_2d(mv, sbase + kVOff + (2 * slot + h) * kHalf, bar(B_VFULL0 + slot), h * 64, y);
           }
         }
         if (!ok) {
@@ -375,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           p.valid = 0;
           return true;
         };
-        for (ItemStream<G> is(plan, blockIdx.x, gridDim.x, b); is.valid() && ok;) {
+        for (ItemStream<G> is(plan, reqx, blockIdx.x, gridDim.x, b); is.valid() && ok;) {
           const Item m = is.next();
           const int nx = 1 + m.has_b;
           for (int t = 0; t < m.n_tiles && ok; ++t, ++n_kv) {
@@ -446,20 +480,24 @@ cudaError_t attention_tc_setup() {
   return cudaFuncSetAttribute(attention_tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
 }
 
-cudaError_t attention_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const PlanHdr* plan,
-                         int64_t kv_rows, int n_q_heads, int n_kv_heads, float scale, __half* o, DevStatus* st,
+cudaError_t attention_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tks,
+                         const CUtensorMap& tvs, const PlanHdr* plan, const int2* reqx, int64_t kv_rows,
+                         int64_t store_rows, int n_q_heads, int n_kv_heads, float scale, __half* o, DevStatus* st,
                          int grid, cudaStream_t s) {
   const int G = n_q_heads / n_kv_heads;
   const float sl2 = scale * 1.4426950408889634f;  // softmax in base 2
   switch (G) {
     case 1:
-      attention_tc_kernel<1><<<grid, kThreads, kSmem, s>>>(tq, tk, tv, plan, kv_rows, n_q_heads, sl2, o, st);
+      attention_tc_kernel<1><<<grid, kThreads, kSmem, s>>>(tq, tk, tv, tks, tvs, plan, reqx, kv_rows, store_rows,
+                                                           n_q_heads, sl2, o, st);
       break;
     case 2:
-      attention_tc_kernel<2><<<grid, kThreads, kSmem, s>>>(tq, tk, tv, plan, kv_rows, n_q_heads, sl2, o, st);
+      attention_tc_kernel<2><<<grid, kThreads, kSmem, s>>>(tq, tk, tv, tks, tvs, plan, reqx, kv_rows, store_rows,
+                                                           n_q_heads, sl2, o, st);
       break;
     case 4:
-      attention_tc_kernel<4><<<grid, kThreads, kSmem, s>>>(tq, tk, tv, plan, kv_rows, n_q_heads, sl2, o, st);
+      attention_tc_kernel<4><<<grid, kThreads, kSmem, s>>>(tq, tk, tv, tks, tvs, plan, reqx, kv_rows, store_rows,
+                                                           n_q_heads, sl2, o, st);
       break;
     default:
       return cudaErrorInvalidValue;

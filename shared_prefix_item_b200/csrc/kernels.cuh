@@ -89,13 +89,24 @@ cudaError_t debug_wait_timeout(DevStatus* st, cudaStream_t s);
 cudaError_t debug_mask(const PlanHdr* plan, int request, uint8_t* out, int64_t tq, cudaStream_t s);
 
 // ---- attention
-cudaError_t attention_f32(const PlanHdr* plan, const float* q, const float* kc, const float* vc, int64_t kv_rows,
-                          int n_q_heads, int n_kv_heads, int hd, float scale, float* o, int max_rows,
-                          cudaStream_t s);
-// tcgen05 attention (fp16 path): items of two 128-slot query sub-tiles, KV tiles of 128 keys
-cudaError_t attention_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const PlanHdr* plan,
-                         int64_t kv_rows, int n_q_heads, int n_kv_heads, float scale, __half* o, DevStatus* st,
+// reqx[r] = {c, s}: request r continues a cached prefix of c tokens whose K/V
+// are rows [s, s + c) (of every KV head) of the layer's KV store; {0, 0}
+// for a request computed from its first token.
+cudaError_t attention_f32(const PlanHdr* plan, const int2* reqx, const float* q, const float* kc, const float* vc,
+                          int64_t kv_rows, const float* ks, const float* vs, int64_t store_rows, int n_q_heads,
+                          int n_kv_heads, int hd, float scale, float* o, int max_rows, cudaStream_t s);
+// tcgen05 attention (fp16 path): items of two 128-slot query sub-tiles, KV
+// tiles of 128 keys; tks / tvs map the layer's KV store
+cudaError_t attention_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tks,
+                         const CUtensorMap& tvs, const PlanHdr* plan, const int2* reqx, int64_t kv_rows,
+                         int64_t store_rows, int n_q_heads, int n_kv_heads, float scale, __half* o, DevStatus* st,
                          int grid, cudaStream_t s);
+// KV store append: for every request r with append[r] = {n, dst} (n > 0),
+// rows [tok0_r, tok0_r + n) of this batch's K/V (every KV head) are copied
+// to store rows [dst, dst + n); row_bytes a multiple of 16
+cudaError_t kv_append(const PlanHdr* plan, const int2* append, const void* kc, const void* vc, int64_t kv_rows,
+                      void* ks, void* vs, int64_t store_rows, int n_kv_heads, int row_bytes, int max_req,
+                      int grid, cudaStream_t s);
 cudaError_t attention_tc_setup();
 int attention_tc_rows_per_item(int group);
 

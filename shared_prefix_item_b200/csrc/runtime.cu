@@ -92,6 +92,19 @@ struct duolm_ctx {
   CUtensorMap tm_xn, tm_oact, tm_h;
   CUtensorMap tm_q3, tm_kc, tm_vc;  // attention operands
 
+  // prefix KV store: per layer [n_kv_heads][n_slots * slot_tokens][head_dim]
+  // for K and for V; slot s of a head starts at row s * slot_tokens
+  void* ks = nullptr;
+  void* vs = nullptr;
+  int n_slots = 0, slot_tokens = 0;
+  int64_t layer_store_elems = 0;  // elements of one layer's K (or V) store
+  std::vector<CUtensorMap> tm_ks, tm_vs;  // per layer (fp16 path)
+  std::vector<int> slot_len;     // valid rows of every slot
+  std::vector<std::pair<int, int>> slot_update;  // (slot, length) once the prepared batch has run
+  int2* reqx = nullptr;          // [cap_R] {cached tokens, first store row}
+  int2* append = nullptr;        // [cap_R] {rows kept, first store row they go to}
+  int2* reqx_host = nullptr;     // pinned staging of both (2 cap_R)
+
   bool prepared = false;
   int64_t n_tokens = 0, n_cand = 0;
   int n_req = 0, branch_len = 1;
@@ -234,8 +247,12 @@ void free_workspace(duolm_ctx* c) {
   dfree(c->ssp);
   dfree(c->scores);
   dfree(c->plan_dev);
+  dfree(c->reqx);
+  dfree(c->append);
   if (c->plan_host) cudaFreeHost(c->plan_host);
   c->plan_host = nullptr;
+  if (c->reqx_host) cudaFreeHost(c->reqx_host);
+  c->reqx_host = nullptr;
   c->cap_T = c->cap_R = c->cap_C = c->cap_I = c->plan_cap = 0;
 }
 
@@ -292,6 +309,11 @@ int reserve_impl(duolm_ctx* ctx, int64_t T, int64_t R, int64_t C) {
   const int64_t pb = plan_bytes_for(T, R, C, I, ctx->num_sms);
   if ((rc = dalloc(ctx, &ctx->plan_dev, pb))) return rc;
   CK(cudaMallocHost(reinterpret_cast<void**>(&ctx->plan_host), pb));
+  if ((rc = dalloc(ctx, &ctx->reqx, R * sizeof(int2)))) return rc;
+  if ((rc = dalloc(ctx, &ctx->append, R * sizeof(int2)))) return rc;
+  CK(cudaMemset(ctx->reqx, 0, R * sizeof(int2)));
+  CK(cudaMemset(ctx->append, 0, R * sizeof(int2)));
+  CK(cudaMallocHost(reinterpret_cast<void**>(&ctx->reqx_host), 2 * R * sizeof(int2)));
   ctx->cap_T = T;
   ctx->cap_R = R;
   ctx->cap_C = C;
@@ -348,6 +370,7 @@ cudaError_t launch_forward(duolm_ctx* c, int n_layers, bool with_head, int64_t* 
   cudaStream_t s = c->stream;
   const int maxT = (int)c->cap_T;
   const int64_t kv_rows = c->cap_T + kKvPad;
+  const int64_t store_rows = (int64_t)c->n_slots * c->slot_tokens;
   const float attn_scale = 1.0f / sqrtf((float)d.head_dim);
   int64_t launches = 0;
   if (c->f16) {
@@ -365,8 +388,17 @@ cudaError_t launch_forward(duolm_ctx* c, int n_layers, bool with_head, int64_t* 
                     kv_rows, kMaxPos, c->gains + L.g_q, c->gains + L.g_k, L.s_qkv, d.rms_eps, c->qd, c->kd,
                     d.n_q_heads, c->ssp, n_slots, inv_d, d.rms_eps};
       LCK(DUOLM_PROF_GEMM_QKV, gemm_tc_qkv(c->tm_xn, L.tm_qkv, d.d, c->qd + 2 * c->kd, plan, qa, c->status, c->gemm_grid, s));
-      LCK(DUOLM_PROF_ATTENTION, attention_tc(c->tm_q3, c->tm_kc, c->tm_vc, plan, kv_rows, d.n_q_heads, d.n_kv_heads,
-                                             attn_scale, static_cast<__half*>(c->o), c->status, c->num_sms, s));
+      // without a store, the batch's own maps stand in for the store maps
+      // (no request has cached tokens then, so no tile reads them)
+      LCK(DUOLM_PROF_ATTENTION,
+          attention_tc(c->tm_q3, c->tm_kc, c->tm_vc, c->ks ? c->tm_ks[l] : c->tm_kc, c->ks ? c->tm_vs[l] : c->tm_vc,
+                       plan, c->reqx, kv_rows, store_rows, d.n_q_heads, d.n_kv_heads, attn_scale,
+                       static_cast<__half*>(c->o), c->status, c->num_sms, s));
+      if (c->ks)
+        LCK(DUOLM_PROF_KV_APPEND, kv_append(plan, c->append, c->kc, c->vc, kv_rows,
+                                            static_cast<__half*>(c->ks) + l * c->layer_store_elems,
+                                            static_cast<__half*>(c->vs) + l * c->layer_store_elems, store_rows,
+                                            d.n_kv_heads, d.head_dim * 2, (int)c->cap_R, 2 * c->num_sms, s));
       LCK(DUOLM_PROF_GEMM_O, gemm_tc_resid(c->tm_oact, L.tm_o, c->qd, d.d, plan,
                                            EpiResidArgs{c->x, d.d, L.s_o, xg, c->gains + L.g_mlp, c->ssp, n_slots},
                                            c->status, c->gemm_grid, s));
@@ -392,9 +424,16 @@ cudaError_t launch_forward(duolm_ctx* c, int n_layers, bool with_head, int64_t* 
       LCK(DUOLM_PROF_GEMM_QKV, qkv_post_f32(plan, c->qkv32, d.n_q_heads, d.n_kv_heads, d.head_dim, c->gains + L.g_q, c->gains + L.g_k,
                        d.rms_eps, c->rope, kMaxPos, static_cast<float*>(c->q), static_cast<float*>(c->kc),
                        static_cast<float*>(c->vc), kv_rows, c->status, maxT, s));
-      LCK(DUOLM_PROF_ATTENTION, attention_f32(plan, static_cast<float*>(c->q), static_cast<float*>(c->kc), static_cast<float*>(c->vc),
-                        kv_rows, d.n_q_heads, d.n_kv_heads, d.head_dim, attn_scale, static_cast<float*>(c->o),
-                        maxT, s));
+      const float* ks = c->ks ? static_cast<const float*>(c->ks) + l * c->layer_store_elems : nullptr;
+      const float* vs = c->vs ? static_cast<const float*>(c->vs) + l * c->layer_store_elems : nullptr;
+      LCK(DUOLM_PROF_ATTENTION, attention_f32(plan, c->reqx, static_cast<float*>(c->q), static_cast<float*>(c->kc),
+                                              static_cast<float*>(c->vc), kv_rows, ks, vs, store_rows, d.n_q_heads,
+                                              d.n_kv_heads, d.head_dim, attn_scale, static_cast<float*>(c->o), maxT,
+                                              s));
+      if (c->ks)
+        LCK(DUOLM_PROF_KV_APPEND, kv_append(plan, c->append, c->kc, c->vc, kv_rows, const_cast<float*>(ks),
+                                            const_cast<float*>(vs), store_rows, d.n_kv_heads, d.head_dim * 4,
+                                            (int)c->cap_R, 2 * c->num_sms, s));
       LCK(DUOLM_PROF_GEMM_O, gemm_simt(static_cast<float*>(c->o), static_cast<const float*>(L.wo), c->x, c->qd, d.d, d.d, true, plan,
                     maxT, s));
       LCK(DUOLM_PROF_RMSNORM, rmsnorm_rows<float>(plan, c->x, d.d, c->gains + L.g_mlp, d.rms_eps, xn, c->status, maxT, s));
@@ -430,10 +469,13 @@ int check_status(duolm_ctx* ctx) {
 }
 
 struct ReqView {
-  const int32_t* prefix;
+  const int32_t* prefix;  // the new prefix tokens (after the cached ones)
   int64_t L;
   const int32_t* branch;  // K * b ids
   int64_t K;
+  int cached;             // prefix tokens already in the slot
+  int slot;               // KV store slot, -1: none
+  int keep;               // new prefix tokens appended to the slot
 };
 
 }  // namespace
@@ -647,8 +689,15 @@ int duolm_reserve(duolm_ctx* ctx, int64_t max_tokens, int64_t max_requests, int6
   return reserve_impl(ctx, max_tokens, max_requests, max_candidates);
 }
 
-int duolm_prepare(duolm_ctx* ctx, int n_requests, const int32_t* prefix_ids, const int64_t* prefix_offsets,
-                  const int32_t* branch_ids, const int64_t* cand_offsets, int branch_len, int mode) {
+}  // extern "C"
+
+namespace {
+
+// duolm_prepare and duolm_prepare_cached.  slot == nullptr: no request
+// continues a cached prefix.
+int prepare_impl(duolm_ctx* ctx, int n_requests, const int32_t* prefix_ids, const int64_t* prefix_offsets,
+                 const int32_t* branch_ids, const int64_t* cand_offsets, int branch_len, int mode,
+                 const int32_t* slot, const int32_t* cached, const int32_t* keep) {
   if (!ctx) return DUOLM_E_ARG;
   ctx->prepared = false;
   if (n_requests < 1 || !prefix_ids || !prefix_offsets || !branch_ids || !cand_offsets)
@@ -659,17 +708,44 @@ int duolm_prepare(duolm_ctx* ctx, int n_requests, const int32_t* prefix_ids, con
     return fail(ctx, DUOLM_E_ARG, "prepare: branch_len %d above %d", branch_len, ctx->rows_per_item);
   if (prefix_offsets[0] != 0 || cand_offsets[0] != 0)
     return fail(ctx, DUOLM_E_OFFSETS, "prepare: offsets must start at 0");
+  if (slot && (!cached || !keep)) return fail(ctx, DUOLM_E_ARG, "prepare: null cached or keep array");
   const int64_t vocab = ctx->desc.vocab, id_end = vocab + ctx->n_items;
   std::vector<ReqView> reqs;
+  std::vector<int> slot_uses(slot ? ctx->n_slots : 0, 0), slot_writers(slot ? ctx->n_slots : 0, 0);
   int64_t n_cand = 0;
   for (int q = 0; q < n_requests; ++q) {
     const int64_t L = prefix_offsets[q + 1] - prefix_offsets[q];
     const int64_t K = cand_offsets[q + 1] - cand_offsets[q];
     if (L < 0 || K < 0) return fail(ctx, DUOLM_E_OFFSETS, "prepare: offsets decrease at request %d", q);
-    if (L == 0 || K == 0) return fail(ctx, DUOLM_E_EMPTY, "prepare: request %d has L=%lld K=%lld", q, (long long)L, (long long)K);
-    if (L + branch_len > kMaxPos)
+    const int sl = slot ? slot[q] : -1;
+    int64_t c = 0, kp = 0;
+    if (sl >= 0) {
+      if (ctx->n_slots == 0) return fail(ctx, DUOLM_E_STATE, "prepare: request %d names slot %d but no KV store is reserved", q, sl);
+      if (sl >= ctx->n_slots) return fail(ctx, DUOLM_E_ARG, "prepare: request %d slot %d (store has %d)", q, sl, ctx->n_slots);
+      if (mode != DUOLM_MODE_MIS) return fail(ctx, DUOLM_E_ARG, "prepare: cached prefixes need the multi-item mode");
+      c = cached[q];
+      kp = keep[q];
+      if (c < 0 || kp < 0 || kp > L)
+        return fail(ctx, DUOLM_E_ARG, "prepare: request %d cached %lld keep %lld of %lld new tokens", q, (long long)c,
+                    (long long)kp, (long long)L);
+      if (c > ctx->slot_len[sl])
+        return fail(ctx, DUOLM_E_STATE, "prepare: request %d reuses %lld tokens of slot %d, which holds %d", q,
+                    (long long)c, sl, ctx->slot_len[sl]);
+      if (c + kp > ctx->slot_tokens)
+        return fail(ctx, DUOLM_E_CAPACITY, "prepare: request %d keeps slot %d rows up to %lld (slot size %d)", q, sl,
+                    (long long)(c + kp), ctx->slot_tokens);
+      ++slot_uses[sl];
+      if (kp > 0) ++slot_writers[sl];
+      if (slot_writers[sl] > 0 && slot_uses[sl] > 1)
+        return fail(ctx, DUOLM_E_ARG, "prepare: slot %d is written by one request of the batch and used by another", sl);
+    } else if (slot && (cached[q] != 0 || keep[q] != 0)) {
+      return fail(ctx, DUOLM_E_ARG, "prepare: request %d has no slot but cached or keep set", q);
+    }
+    if ((L == 0 && c == 0) || K == 0)
+      return fail(ctx, DUOLM_E_EMPTY, "prepare: request %d has L=%lld K=%lld", q, (long long)(c + L), (long long)K);
+    if (c + L + branch_len > kMaxPos)
       return fail(ctx, DUOLM_E_CAPACITY, "prepare: request %d needs positions up to %lld (limit %d)", q,
-                  (long long)(L + branch_len), kMaxPos);
+                  (long long)(c + L + branch_len), kMaxPos);
     const int32_t* pre = prefix_ids + prefix_offsets[q];
     const int32_t* br = branch_ids + cand_offsets[q] * branch_len;
     for (int64_t i = 0; i < L; ++i)
@@ -681,9 +757,9 @@ int duolm_prepare(duolm_ctx* ctx, int n_requests, const int32_t* prefix_ids, con
         return fail(ctx, DUOLM_E_ID, "prepare: request %d branch token %lld has id %d (valid: 0..%lld)", q,
                     (long long)i, br[i], (long long)id_end - 1);
     if (mode == DUOLM_MODE_MIS) {
-      reqs.push_back(ReqView{pre, L, br, K});
+      reqs.push_back(ReqView{pre, L, br, K, (int)c, sl, (int)kp});
     } else {
-      for (int64_t c = 0; c < K; ++c) reqs.push_back(ReqView{pre, L, br + c * branch_len, 1});
+      for (int64_t j = 0; j < K; ++j) reqs.push_back(ReqView{pre, L, br + j * branch_len, 1, 0, -1, 0});
     }
     n_cand += K;
   }
@@ -716,21 +792,31 @@ int duolm_prepare(duolm_ctx* ctx, int n_requests, const int32_t* prefix_ids, con
   int32_t* treq = reinterpret_cast<int32_t*>(base + hdr.off_treq);
   int4* rq = reinterpret_cast<int4*>(base + hdr.off_req);
   int32_t* cand = reinterpret_cast<int32_t*>(base + hdr.off_cand);
+  int2* rx = ctx->reqx_host;               // {cached, first store row}
+  int2* ap = ctx->reqx_host + ctx->cap_R;  // {rows kept, store row of the first}
   ctx->req_host.assign(R, int4{0, 0, 0, 0});
+  ctx->slot_update.clear();
   int64_t t = 0, c = 0;
   for (int64_t r = 0; r < R; ++r) {
     const ReqView& v = reqs[r];
-    rq[r] = int4{(int)t, (int)v.L, (int)v.K, (int)c};
+    // request-local indices count from the first cached token: the prefix
+    // is c + L tokens long, the batch holds indices c .. c + L - 1
+    const int64_t Lt = v.cached + v.L;
+    rq[r] = int4{(int)t, (int)Lt, (int)v.K, (int)c};
     ctx->req_host[r] = rq[r];
+    const int row0 = v.slot >= 0 ? v.slot * ctx->slot_tokens : 0;
+    rx[r] = int2{v.cached, row0};
+    ap[r] = int2{v.keep, row0 + v.cached};
+    if (v.slot >= 0 && v.keep > 0) ctx->slot_update.push_back({v.slot, v.cached + v.keep});
     for (int64_t i = 0; i < v.L; ++i, ++t) {
       ids[t] = v.prefix[i];
-      pos[t] = (int32_t)i;  // prefix token i at position i
+      pos[t] = (int32_t)(v.cached + i);  // prefix token i at its position in the whole prefix
       treq[t] = (int32_t)r;
     }
     for (int64_t j = 0; j < v.K; ++j) {
       for (int64_t i = 0; i < branch_len; ++i, ++t) {
         ids[t] = v.branch[j * branch_len + i];
-        pos[t] = (int32_t)(v.L + i);  // every branch at logical position L (+ i inside the branch)
+        pos[t] = (int32_t)(Lt + i);  // every branch at logical position L (+ i inside the branch)
         treq[t] = (int32_t)r;
       }
       cand[c++] = (int32_t)(t - 1);  // the branch's last token is scored
@@ -740,29 +826,35 @@ int duolm_prepare(duolm_ctx* ctx, int n_requests, const int32_t* prefix_ids, con
   // stay together so that the CTAs running them at the same time share that
   // head's prefix K/V through L2; groups go most expensive first, and inside
   // a group branch items come first, then prefix items from the last rows.
+  // A request's query rows start at its cached length c; its key tiles are
+  // ceil(c / 128) store tiles, then tiles of 128 from c.
   int64_t n_items = 0;
   if (ctx->f16) {
     const int Rw = ctx->rows_per_item;
     const int per = (Rw / branch_len) * branch_len;
     const int key_tile = 128;
+    auto prefix_tiles = [&](int cached, int kend) -> int64_t {
+      return (cached + key_tile - 1) / key_tile + (kend - cached + key_tile - 1) / key_tile;
+    };
     std::vector<std::pair<int64_t, int64_t>> groups;  // (cost in key tiles, request * n_kv_heads + kvh)
     groups.reserve((size_t)R * ctx->desc.n_kv_heads);
     for (int64_t r = 0; r < R; ++r) {
-      const int L = rq[r].y, K = rq[r].z;
+      const int L = rq[r].y, K = rq[r].z, cr = rx[r].x;
       int64_t cost = 0;
-      for (int row0 = 0; row0 < L; row0 += Rw) cost += (std::min(row0 + Rw, L) + key_tile - 1) / key_tile;
-      cost += (int64_t)((K * branch_len + per - 1) / per) * ((L + key_tile - 1) / key_tile + 1);
+      for (int row0 = cr; row0 < L; row0 += Rw) cost += prefix_tiles(cr, std::min(row0 + Rw, L));
+      cost += (int64_t)((K * branch_len + per - 1) / per) * (prefix_tiles(cr, L) + 1);
       for (int kvh = 0; kvh < ctx->desc.n_kv_heads; ++kvh) groups.push_back({cost, r * ctx->desc.n_kv_heads + kvh});
     }
     std::stable_sort(groups.begin(), groups.end(), [](const auto& a, const auto& b) { return a.first > b.first; });
     int4* it = reinterpret_cast<int4*>(base + hdr.off_items);
     for (const auto& g : groups) {
       const int r = (int)(g.second / ctx->desc.n_kv_heads), kvh = (int)(g.second % ctx->desc.n_kv_heads);
-      const int L = rq[r].y, K = rq[r].z;
-      const int64_t need = (K * branch_len + per - 1) / per + (L + Rw - 1) / Rw;
+      const int L = rq[r].y, K = rq[r].z, cr = rx[r].x;
+      const int64_t need = (K * branch_len + per - 1) / per + (L - cr + Rw - 1) / Rw;
       if (n_items + need > ctx->cap_I) return fail(ctx, DUOLM_E_CAPACITY, "prepare: work list overflow");
       for (int row0 = 0; row0 < K * branch_len; row0 += per) it[n_items++] = int4{r, kvh, 1, row0};
-      for (int row0 = ((L - 1) / Rw) * Rw; row0 >= 0; row0 -= Rw) it[n_items++] = int4{r, kvh, 0, row0};
+      if (L > cr)
+        for (int row0 = cr + ((L - cr - 1) / Rw) * Rw; row0 >= cr; row0 -= Rw) it[n_items++] = int4{r, kvh, 0, row0};
     }
     // Each CTA runs the items the greedy list schedule gives it: in list
     // order, an item goes to the CTA with the least work so far.  The
@@ -779,10 +871,10 @@ int duolm_prepare(duolm_ctx* ctx, int n_requests, const int32_t* prefix_ids, con
       const int half_rows = Rw / 2;  // rows of one query sub-tile
       for (int64_t i = 0; i < n_items; ++i) {
         const int4 m = it[i];
-        const int L = rq[m.x].y, K = rq[m.x].z;
+        const int L = rq[m.x].y, K = rq[m.x].z, cr = rx[m.x].x;
         const int nrows = m.z ? std::min(per, K * branch_len - m.w) : std::min(Rw, L - m.w);
         const int kend = m.z ? L : std::min(m.w + Rw, L);
-        const int64_t tiles = (kend + key_tile - 1) / key_tile + (m.z ? (nrows + key_tile - 1) / key_tile : 0);
+        const int64_t tiles = prefix_tiles(cr, kend) + (m.z ? (nrows + key_tile - 1) / key_tile : 0);
         const int64_t cost = 10 * tiles + (nrows > half_rows ? 2 * tiles : 0) + 5;
         auto top = load.top();
         load.pop();
@@ -805,6 +897,8 @@ int duolm_prepare(duolm_ctx* ctx, int n_requests, const int32_t* prefix_ids, con
                                      : hdr.off_items + align16(n_items * 16);
   memcpy(base, &hdr, sizeof hdr);
   CK(cudaMemcpyAsync(ctx->plan_dev, base, bytes, cudaMemcpyHostToDevice, ctx->stream));
+  CK(cudaMemcpyAsync(ctx->reqx, rx, R * sizeof(int2), cudaMemcpyHostToDevice, ctx->stream));
+  CK(cudaMemcpyAsync(ctx->append, ap, R * sizeof(int2), cudaMemcpyHostToDevice, ctx->stream));
   CK(cudaEventRecord(ctx->plan_ev, ctx->stream));
   ctx->hdr = hdr;
   ctx->n_tokens = T;
@@ -815,10 +909,94 @@ int duolm_prepare(duolm_ctx* ctx, int n_requests, const int32_t* prefix_ids, con
   return 0;
 }
 
+}  // namespace
+
+extern "C" {
+
+int duolm_prepare(duolm_ctx* ctx, int n_requests, const int32_t* prefix_ids, const int64_t* prefix_offsets,
+                  const int32_t* branch_ids, const int64_t* cand_offsets, int branch_len, int mode) {
+  return prepare_impl(ctx, n_requests, prefix_ids, prefix_offsets, branch_ids, cand_offsets, branch_len, mode,
+                      nullptr, nullptr, nullptr);
+}
+
+int duolm_prepare_cached(duolm_ctx* ctx, int n_requests, const int32_t* prefix_ids, const int64_t* prefix_offsets,
+                         const int32_t* branch_ids, const int64_t* cand_offsets, int branch_len, const int32_t* slot,
+                         const int32_t* cached, const int32_t* keep) {
+  if (!ctx) return DUOLM_E_ARG;
+  if (!slot) {
+    ctx->prepared = false;
+    return fail(ctx, DUOLM_E_ARG, "prepare_cached: null slot array");
+  }
+  return prepare_impl(ctx, n_requests, prefix_ids, prefix_offsets, branch_ids, cand_offsets, branch_len,
+                      DUOLM_MODE_MIS, slot, cached, keep);
+}
+
+int duolm_kv_store_reserve(duolm_ctx* ctx, int n_slots, int slot_tokens) {
+  if (!ctx) return DUOLM_E_ARG;
+  if (n_slots < 0 || slot_tokens < 0 || (n_slots > 0 && slot_tokens < 1) || slot_tokens > kMaxPos)
+    return fail(ctx, DUOLM_E_ARG, "kv_store_reserve: %d slots of %d tokens", n_slots, slot_tokens);
+  const auto& d = ctx->desc;
+  const int64_t rows = (int64_t)n_slots * slot_tokens;
+  if (rows * d.n_kv_heads + 256 > INT32_MAX)  // TMA row coordinates are int32
+    return fail(ctx, DUOLM_E_CAPACITY, "kv_store_reserve: %lld rows per layer", (long long)(rows * d.n_kv_heads));
+  CK(cudaSetDevice(ctx->device));
+  CK(cudaStreamSynchronize(ctx->stream));
+  invalidate_graph(ctx);
+  ctx->prepared = false;
+  dfree(ctx->ks);
+  dfree(ctx->vs);
+  ctx->tm_ks.clear();
+  ctx->tm_vs.clear();
+  ctx->slot_len.clear();
+  ctx->slot_update.clear();
+  ctx->n_slots = ctx->slot_tokens = 0;
+  ctx->layer_store_elems = 0;
+  if (n_slots == 0) return 0;
+  const int64_t es = ctx->f16 ? 2 : 4;
+  const int64_t elems = rows * d.n_kv_heads * d.head_dim;
+  const int64_t bytes = elems * d.n_layers * es;
+  int rc;
+  if ((rc = dalloc(ctx, &ctx->ks, bytes)) || (rc = dalloc(ctx, &ctx->vs, bytes))) {
+    dfree(ctx->ks);
+    dfree(ctx->vs);
+    return rc;
+  }
+  // zero rows are finite: a store tile's masked rows never hold NaN
+  CK(cudaMemset(ctx->ks, 0, bytes));
+  CK(cudaMemset(ctx->vs, 0, bytes));
+  if (ctx->f16) {
+    ctx->tm_ks.resize(d.n_layers);
+    ctx->tm_vs.resize(d.n_layers);
+    char e[256];
+    for (int l = 0; l < d.n_layers; ++l)
+      if (!make_tmap_f16_2d(&ctx->tm_ks[l], static_cast<__half*>(ctx->ks) + l * elems, 128,
+                            (uint64_t)d.n_kv_heads * rows, 64, 128, e, sizeof e) ||
+          !make_tmap_f16_2d(&ctx->tm_vs[l], static_cast<__half*>(ctx->vs) + l * elems, 128,
+                            (uint64_t)d.n_kv_heads * rows, 64, 128, e, sizeof e)) {
+        dfree(ctx->ks);
+        dfree(ctx->vs);
+        return fail(ctx, DUOLM_E_CUDA, "%s", e);
+      }
+  }
+  ctx->n_slots = n_slots;
+  ctx->slot_tokens = slot_tokens;
+  ctx->layer_store_elems = elems;
+  ctx->slot_len.assign(n_slots, 0);
+  return 0;
+}
+
+int duolm_kv_slot_length(const duolm_ctx* ctx, int slot) {
+  if (!ctx || slot < 0 || slot >= ctx->n_slots) return DUOLM_E_ARG;
+  return ctx->slot_len[slot];
+}
+
 int duolm_execute(duolm_ctx* ctx) {
   if (!ctx) return DUOLM_E_ARG;
   if (!ctx->prepared) return fail(ctx, DUOLM_E_STATE, "execute: nothing prepared");
   CK(cudaSetDevice(ctx->device));
+  // the slots this batch appends to hold its rows once the launches below
+  // have run (work on the same stream sees them)
+  for (const auto& u : ctx->slot_update) ctx->slot_len[u.first] = u.second;
   if (!ctx->use_graph) {
     CK(launch_forward(ctx, ctx->desc.n_layers, true, &ctx->launches));
     return 0;
@@ -909,6 +1087,19 @@ int duolm_score(duolm_ctx* ctx, int n_requests, const int32_t* prefix_ids, const
   return duolm_sync(ctx);
 }
 
+int duolm_score_cached(duolm_ctx* ctx, int n_requests, const int32_t* prefix_ids, const int64_t* prefix_offsets,
+                       const int32_t* branch_ids, const int64_t* cand_offsets, int branch_len, const int32_t* slot,
+                       const int32_t* cached, const int32_t* keep, float* scores_out) {
+  if (!ctx) return DUOLM_E_ARG;
+  if (!scores_out) return fail(ctx, DUOLM_E_ARG, "score_cached: null scores_out");
+  int rc = duolm_prepare_cached(ctx, n_requests, prefix_ids, prefix_offsets, branch_ids, cand_offsets, branch_len,
+                                slot, cached, keep);
+  if (!rc) rc = duolm_execute(ctx);
+  if (rc) return rc;
+  CK(cudaMemcpyAsync(scores_out, ctx->scores, ctx->n_cand * 4, cudaMemcpyDeviceToHost, ctx->stream));
+  return duolm_sync(ctx);
+}
+
 int duolm_set_graph(duolm_ctx* ctx, int enabled) {
   if (!ctx) return DUOLM_E_ARG;
   ctx->use_graph = enabled != 0;
@@ -925,6 +1116,8 @@ void duolm_destroy(duolm_ctx* ctx) {
   if (ctx->stream) cudaStreamSynchronize(ctx->stream);
   invalidate_graph(ctx);
   free_workspace(ctx);
+  dfree(ctx->ks);
+  dfree(ctx->vs);
   for (auto& L : ctx->layers) {
     dfree(L.wqkv);
     dfree(L.wo);

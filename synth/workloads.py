@@ -159,6 +159,14 @@ class Workload:
         coff[1:] = np.cumsum([r.K for r in self.requests])
         return prefix, poff, branch, coff
 
+    def history_offsets(self, q: int) -> List[int]:
+        """Prefix offset of each history item of request q (its marker)."""
+        o, out = len(self.template.instr), []
+        for f in self.requests[q].feedback:
+            out.append(o)
+            o += 1 + self.m + len(f)
+        return out
+
     def records(self):
         """The requests as records (item ids and feedback tokens, no ids of
         the ranker's sequence): history items + offsets, feedback tokens +
