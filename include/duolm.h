@@ -349,7 +349,8 @@ int duolm_debug_residual(duolm_ctx *ctx, int n_layers, float *x_out);
 /* Copy the device item table out (host uint16 [n_items][d]).  Synchronous. */
 int duolm_debug_table(duolm_ctx *ctx, uint16_t *out, int64_t n_items);
 
-/* Bytes the last duolm_prepare copied host -> device (the packed plan). */
+/* Bytes the last duolm_prepare / duolm_prepare_cached copied host ->
+ * device (the packed plan and the per-request cached-prefix records). */
 int64_t duolm_plan_bytes(const duolm_ctx *ctx);
 
 /*

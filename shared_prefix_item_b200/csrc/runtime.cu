@@ -1180,8 +1180,9 @@ int duolm_debug_residual(duolm_ctx* ctx, int n_layers, float* x_out) {
 
 int64_t duolm_plan_bytes(const duolm_ctx* ctx) {
   if (!ctx || !ctx->prepared) return 0;
-  return ctx->hdr.att_ctas ? ctx->hdr.off_cta + align16((int64_t)(ctx->hdr.att_ctas + 1) * 4)
-                           : ctx->hdr.off_items + align16((int64_t)ctx->hdr.n_items * 16);
+  const int64_t plan = ctx->hdr.att_ctas ? ctx->hdr.off_cta + align16((int64_t)(ctx->hdr.att_ctas + 1) * 4)
+                                         : ctx->hdr.off_items + align16((int64_t)ctx->hdr.n_items * 16);
+  return plan + 2 * (int64_t)ctx->n_req * (int64_t)sizeof(int2);  // + the cached-prefix and append records
 }
 
 int duolm_debug_gemm(duolm_ctx* ctx, int layer, int which, const uint16_t* a, float* out) {
