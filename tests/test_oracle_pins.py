@@ -240,6 +240,24 @@ def test_causal_prefix():
     assert not np.array_equal(layers[-1, 30:], layers2[-1, 30:])
 
 
+def test_prefix_rows_of_a_shorter_call_equal_those_of_the_whole_sequence():
+    """The reading behind prefix KV reuse: in the packed multi-item layout a
+    prefix row's residual at every layer (hence its K/V) is the same whether
+    the call held the prefix up to some cut with its own candidates, or the
+    whole prefix with other candidates."""
+    m = _tiny_model()
+    tab = _tiny_table(m)
+    req = W.tiny().requests[0]
+    c = 29
+    short = R.mis_layout(req.prefix_ids[:c], req.branch_ids[:3])
+    full = R.mis_layout(req.prefix_ids, req.branch_ids[3:])
+    _, ls = R.forward(m, tab, short, want_layers=True)
+    _, lf = R.forward(m, tab, full, want_layers=True)
+    assert np.array_equal(ls[:, :c], lf[:, :c])
+    # the branches of the short call sit at position c, those of the whole one at L
+    assert short.pos[c] == c and full.pos[req.L] == req.L
+
+
 # --------------------------------------------------------------------------
 # whole-model special cases with hand-computable results
 # --------------------------------------------------------------------------
