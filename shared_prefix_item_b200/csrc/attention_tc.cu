@@ -469,7 +469,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 int attention_tc_rows_per_item(int group) { return 2 * kSub / group; }
-int attention_tc_smem_bytes() { return kSmem; }
 
 cudaError_t attention_tc_setup() {
   cudaError_t e;

@@ -603,10 +603,6 @@ bool make_tmap_f16_3d(CUtensorMap* map, const void* base, const uint64_t dims[3]
   return true;
 }
 
-int gemm_tc_smem_bytes(int) {
-  return std::max(TcCfg<256, EpiResid>::SMEM, std::max(TcCfg<256, EpiSwiglu>::SMEM, TcCfg<256, EpiQkv>::SMEM));
-}
-
 cudaError_t gemm_tc_setup() {
   cudaError_t e;
   if ((e = cudaFuncSetAttribute(gemm_tc_kernel<256, EpiResid>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -51,7 +51,6 @@ bool make_tmap_f16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64
                       uint32_t box_outer, char* err, size_t errlen);
 bool make_tmap_f16_3d(CUtensorMap* map, const void* base, const uint64_t dims[3], const uint64_t strides_bytes[2],
                       const uint32_t box[3], char* err, size_t errlen);
-int gemm_tc_smem_bytes(int bn);
 cudaError_t gemm_tc_setup();
 cudaError_t gemm_tc_resid(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
                           EpiResidArgs e, DevStatus* st, int grid, cudaStream_t s);
