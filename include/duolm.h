@@ -346,6 +346,21 @@ int duolm_debug_mask(duolm_ctx *ctx, int request, uint8_t *out);
  * gives the looked-up rows.  Synchronous. */
 int duolm_debug_residual(duolm_ctx *ctx, int n_layers, float *x_out);
 
+/*
+ * The attention work list duolm_prepare builds on the tensor-core path, for
+ * a batch described by its request sizes alone (host only, no context, no
+ * GPU).  Request r has a whole prefix of L[r] tokens, cached[r] of them from
+ * the prefix KV store, and K[r] candidates of branch_len tokens.  Writes
+ * items [cap_items][4] = {request, KV head, kind (1: whole candidate
+ * branches from branch row `row`; 0: prefix rows from `row`), row} and
+ * cta_off [n_ctas + 1] (CTA c runs items cta_off[c] .. cta_off[c+1] - 1).
+ * Returns the item count, DUOLM_E_CAPACITY when above cap_items, DUOLM_E_ARG.
+ */
+int64_t duolm_debug_attention_plan(int n_requests, const int32_t *L, const int32_t *K,
+                                   const int32_t *cached, int branch_len, int n_kv_heads,
+                                   int rows_per_item, int n_ctas, int32_t *items, int64_t cap_items,
+                                   int32_t *cta_off);
+
 /* Copy the device item table out (host uint16 [n_items][d]).  Synchronous. */
 int duolm_debug_table(duolm_ctx *ctx, uint16_t *out, int64_t n_items);
 

@@ -7,8 +7,8 @@ fail loudly if it has not been built (``python -m
 shared_prefix_item_b200.build``); importing the ``build`` submodule does not
 load it.
 """
-_PUBLIC = ("DTYPE_BF16", "DTYPE_FP32", "MODE_INDEPENDENT", "MODE_MIS", "DuolmError", "Ranker", "compile_requests", "lib",
-           "lib_path")
+_PUBLIC = ("DTYPE_BF16", "DTYPE_FP32", "MODE_INDEPENDENT", "MODE_MIS", "DuolmError", "Ranker", "attention_plan",
+           "compile_requests", "lib", "lib_path")
 
 
 def __getattr__(name):

@@ -76,6 +76,7 @@ def _load():
         "duolm_embedding_rho_static": (I, [VP, I, I64, I, VP, VP]),
         "duolm_gather": (I, [VP, VP, I64, VP, VP, VP]),
         "duolm_compile": (I, [P(Template), I, VP, VP, VP, VP, VP, VP, I64, I, VP, I64, VP, VP, I64]),
+        "duolm_debug_attention_plan": (I64, [I, VP, VP, VP, I, I, I, I, VP, I64, VP]),
         "duolm_kv_store_reserve": (I, [VP, I, I]),
         "duolm_kv_slot_length": (I, [VP, I]),
         "duolm_prepare_cached": (I, [VP, I, VP, VP, VP, VP, I, VP, VP, VP]),
@@ -126,6 +127,21 @@ def compile_requests(vocab: int, marker: int, m: int, instr, header, branch_head
     if rc != 0:
         raise DuolmError(rc, lib.duolm_last_error(None).decode())
     return prefix[:int(poff[-1])], poff, branch[:int(co[-1]) * b], co, b
+
+
+def attention_plan(L, K, cached, branch_len: int, n_kv_heads: int, rows_per_item: int, n_ctas: int):
+    """duolm_debug_attention_plan: (items [n][4], cta_off [n_ctas + 1])."""
+    Ls, Ks, cs = (np.ascontiguousarray(x, np.int32) for x in (L, K, cached))
+    per = (rows_per_item // branch_len) * branch_len
+    cap = int(n_kv_heads * sum((k * branch_len + per - 1) // per + (l - c + rows_per_item - 1) // rows_per_item
+                               for l, k, c in zip(Ls, Ks, cs)))
+    items = np.zeros((max(cap, 1), 4), np.int32)
+    cta = np.zeros(n_ctas + 1, np.int32)
+    n = lib.duolm_debug_attention_plan(len(Ls), _p(Ls), _p(Ks), _p(cs), int(branch_len), int(n_kv_heads),
+                                       int(rows_per_item), int(n_ctas), _p(items), cap, _p(cta))
+    if n < 0:
+        raise DuolmError(int(n), "duolm_debug_attention_plan")
+    return items[:n], cta
 
 
 def _arr(a, dtype) -> np.ndarray:

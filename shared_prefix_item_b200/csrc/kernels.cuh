@@ -107,6 +107,12 @@ cudaError_t kv_append(const PlanHdr* plan, const int2* append, const void* kc, c
                       void* ks, void* vs, int64_t store_rows, int n_kv_heads, int row_bytes, int max_req,
                       int grid, cudaStream_t s);
 cudaError_t attention_tc_setup();
+// Host: the batch's attention work list {request, KV head, kind (1 branch,
+// 0 prefix), first query row} (req: {tok0, whole prefix L, K, -}; reqx: as
+// above) and the CTA ranges of its greedy list schedule (cta_off[n_ctas + 1]).
+// Returns the item count, or -1 above cap_items.
+int64_t plan_attention(const int4* req, const int2* reqx, int64_t R, int n_kv_heads, int rows_per_item,
+                       int branch_len, int n_ctas, int64_t cap_items, int4* items, int32_t* cta_off);
 int attention_tc_rows_per_item(int group);
 
 }  // namespace duolm

@@ -13,7 +13,6 @@
 #include <cstring>
 #include <string>
 #include <thread>
-#include <queue>
 #include <vector>
 
 #include "common.cuh"
@@ -822,75 +821,17 @@ int prepare_impl(duolm_ctx* ctx, int n_requests, const int32_t* prefix_ids, cons
       cand[c++] = (int32_t)(t - 1);  // the branch's last token is scored
     }
   }
-  // attention work items (fp16 path).  The items of one (request, KV head)
-  // stay together so that the CTAs running them at the same time share that
-  // head's prefix K/V through L2; groups go most expensive first, and inside
-  // a group branch items come first, then prefix items from the last rows.
-  // A request's query rows start at its cached length c; its key tiles are
-  // ceil(c / 128) store tiles, then tiles of 128 from c.
+  // attention work list and its CTA ranges (fp16 path)
   int64_t n_items = 0;
   if (ctx->f16) {
-    const int Rw = ctx->rows_per_item;
-    const int per = (Rw / branch_len) * branch_len;
-    const int key_tile = 128;
-    auto prefix_tiles = [&](int cached, int kend) -> int64_t {
-      return (cached + key_tile - 1) / key_tile + (kend - cached + key_tile - 1) / key_tile;
-    };
-    std::vector<std::pair<int64_t, int64_t>> groups;  // (cost in key tiles, request * n_kv_heads + kvh)
-    groups.reserve((size_t)R * ctx->desc.n_kv_heads);
-    for (int64_t r = 0; r < R; ++r) {
-      const int L = rq[r].y, K = rq[r].z, cr = rx[r].x;
-      int64_t cost = 0;
-      for (int row0 = cr; row0 < L; row0 += Rw) cost += prefix_tiles(cr, std::min(row0 + Rw, L));
-      cost += (int64_t)((K * branch_len + per - 1) / per) * (prefix_tiles(cr, L) + 1);
-      for (int kvh = 0; kvh < ctx->desc.n_kv_heads; ++kvh) groups.push_back({cost, r * ctx->desc.n_kv_heads + kvh});
-    }
-    std::stable_sort(groups.begin(), groups.end(), [](const auto& a, const auto& b) { return a.first > b.first; });
-    int4* it = reinterpret_cast<int4*>(base + hdr.off_items);
-    for (const auto& g : groups) {
-      const int r = (int)(g.second / ctx->desc.n_kv_heads), kvh = (int)(g.second % ctx->desc.n_kv_heads);
-      const int L = rq[r].y, K = rq[r].z, cr = rx[r].x;
-      const int64_t need = (K * branch_len + per - 1) / per + (L - cr + Rw - 1) / Rw;
-      if (n_items + need > ctx->cap_I) return fail(ctx, DUOLM_E_CAPACITY, "prepare: work list overflow");
-      for (int row0 = 0; row0 < K * branch_len; row0 += per) it[n_items++] = int4{r, kvh, 1, row0};
-      if (L > cr)
-        for (int row0 = cr + ((L - cr - 1) / Rw) * Rw; row0 >= cr; row0 -= Rw) it[n_items++] = int4{r, kvh, 0, row0};
-    }
-    // Each CTA runs the items the greedy list schedule gives it: in list
-    // order, an item goes to the CTA with the least work so far.  The
-    // estimated cost of an item is its key tiles, +20% when its second
-    // query sub-tile is in use (the two sub-tiles run side by side), plus
-    // half a tile for starting it.  Items stay in list order within a CTA and
-    // CTAs advance through the list at about the same pace, so the items of
-    // one (request, KV head) still run close together in time.
     const int G = ctx->num_sms;
-    std::vector<int> owner((size_t)n_items);
-    {
-      std::priority_queue<std::pair<int64_t, int>, std::vector<std::pair<int64_t, int>>, std::greater<>> load;
-      for (int g = 0; g < G; ++g) load.push({0, g});
-      const int half_rows = Rw / 2;  // rows of one query sub-tile
-      for (int64_t i = 0; i < n_items; ++i) {
-        const int4 m = it[i];
-        const int L = rq[m.x].y, K = rq[m.x].z, cr = rx[m.x].x;
-        const int nrows = m.z ? std::min(per, K * branch_len - m.w) : std::min(Rw, L - m.w);
-        const int kend = m.z ? L : std::min(m.w + Rw, L);
-        const int64_t tiles = prefix_tiles(cr, kend) + (m.z ? (nrows + key_tile - 1) / key_tile : 0);
-        const int64_t cost = 10 * tiles + (nrows > half_rows ? 2 * tiles : 0) + 5;
-        auto top = load.top();
-        load.pop();
-        owner[i] = top.second;
-        load.push({top.first + cost, top.second});
-      }
-    }
-    std::vector<int4> listed(it, it + n_items);
+    std::vector<int32_t> cta_range((size_t)G + 1);
+    n_items = plan_attention(rq, rx, R, ctx->desc.n_kv_heads, ctx->rows_per_item, branch_len, G, ctx->cap_I,
+                             reinterpret_cast<int4*>(base + hdr.off_items), cta_range.data());
+    if (n_items < 0) return fail(ctx, DUOLM_E_CAPACITY, "prepare: work list overflow");
     hdr.att_ctas = G;
     hdr.off_cta = hdr.off_items + align16(n_items * 16);
-    int32_t* cta_off = reinterpret_cast<int32_t*>(base + hdr.off_cta);
-    std::fill(cta_off, cta_off + G + 1, 0);
-    for (int64_t i = 0; i < n_items; ++i) ++cta_off[owner[i] + 1];
-    for (int g = 0; g < G; ++g) cta_off[g + 1] += cta_off[g];
-    std::vector<int32_t> fill(cta_off, cta_off + G);
-    for (int64_t i = 0; i < n_items; ++i) it[fill[owner[i]]++] = listed[i];
+    memcpy(base + hdr.off_cta, cta_range.data(), (size_t)(G + 1) * 4);
   }
   hdr.n_items = (int32_t)n_items;
   const int64_t bytes = hdr.att_ctas ? hdr.off_cta + align16((int64_t)(hdr.att_ctas + 1) * 4)
