@@ -271,6 +271,27 @@ int duolm_compile(const duolm_template *tpl, int n_requests, const int64_t *hist
                   int64_t branch_capacity);
 
 /*
+ * duolm_compile for requests that continue a prefix in the KV store
+ * (incremental history append, see duolm_prepare_cached).  hist_cached[r]
+ * (host, n_requests entries): -1 for a request that does not use the store
+ * (compiled whole; cached_out 0, keep_out 0); h >= 0 when its slot holds the
+ * instruction and its first h history items (h = 0: the slot is empty).
+ * Only the rest is compiled: for h > 0 the prefix is history items h.. and
+ * the header, for h = 0 the instruction, every history item and the header.
+ * cached_out[r] receives the tokens the slot holds (the instruction and the
+ * first h items; 0 for h = 0), keep_out[r] the new prefix tokens to append
+ * (everything but the header), both ready for duolm_prepare_cached.
+ * Errors as duolm_compile; DUOLM_E_ARG also for h outside -1..items.
+ */
+int duolm_compile_append(const duolm_template *tpl, int n_requests, const int64_t *hist_items,
+                         const int64_t *hist_offsets, const int32_t *feedback,
+                         const int64_t *feedback_offsets, const int64_t *cand_items,
+                         const int64_t *cand_offsets, int64_t n_items, int n_threads,
+                         const int32_t *hist_cached, int32_t *prefix_ids, int64_t prefix_capacity,
+                         int64_t *prefix_offsets, int32_t *branch_ids, int64_t branch_capacity,
+                         int32_t *cached_out, int32_t *keep_out);
+
+/*
  * duolm_gather -- the hot path's first step alone: the virtual-id gather of
  * the ranker's inputs (DuoLM summary page, 方法步骤详情 step 3: an id below
  * the vocabulary V reads the embedding, id V + i reads row i of the FP16 item

@@ -76,6 +76,8 @@ def _load():
         "duolm_embedding_rho_static": (I, [VP, I, I64, I, VP, VP]),
         "duolm_gather": (I, [VP, VP, I64, VP, VP, VP]),
         "duolm_compile": (I, [P(Template), I, VP, VP, VP, VP, VP, VP, I64, I, VP, I64, VP, VP, I64]),
+        "duolm_compile_append": (I, [P(Template), I, VP, VP, VP, VP, VP, VP, I64, I, VP, VP, I64, VP, VP, I64, VP,
+                                     VP]),
         "duolm_debug_attention_plan": (I64, [I, VP, VP, VP, I, I, I, I, VP, I64, VP]),
         "duolm_kv_store_reserve": (I, [VP, I, I]),
         "duolm_kv_slot_length": (I, [VP, I]),
@@ -105,10 +107,14 @@ def embedding_rho_static(embed_dev: int, dtype: int, vocab: int, d: int, rho_out
 
 
 def compile_requests(vocab: int, marker: int, m: int, instr, header, branch_header, hist_items, hist_offsets,
-                     feedback, feedback_offsets, cand_items, cand_offsets, n_items: int, n_threads: int = 0):
+                     feedback, feedback_offsets, cand_items, cand_offsets, n_items: int, n_threads: int = 0,
+                     hist_cached=None):
     """duolm_compile: request records -> (prefix_ids, prefix_offsets,
     branch_ids, cand_offsets, branch_len), host arrays in the layout
-    duolm_prepare / duolm_score take."""
+    duolm_prepare / duolm_score take.  With hist_cached (per request: -1, or
+    the history items its KV slot already holds), duolm_compile_append:
+    the result also carries the cached and keep arrays of
+    duolm_prepare_cached."""
     ins, hdr, bh = (np.ascontiguousarray(x, np.int32) for x in (instr, header, branch_header))
     tpl = Template(int(vocab), int(marker), int(m), ins.ctypes.data, len(ins), hdr.ctypes.data, len(hdr),
                    bh.ctypes.data, len(bh))
@@ -122,11 +128,20 @@ def compile_requests(vocab: int, marker: int, m: int, instr, header, branch_head
     prefix = np.empty(max(cap, 1), np.int32)
     poff = np.empty(R + 1, np.int64)
     branch = np.empty(max(int(co[-1]) * b, 1), np.int32)
-    rc = lib.duolm_compile(ctypes.byref(tpl), R, _p(hi), _p(ho), _p(fb), _p(fo), _p(ci), _p(co), int(n_items),
-                           int(n_threads), _p(prefix), prefix.size, _p(poff), _p(branch), branch.size)
+    if hist_cached is None:
+        rc = lib.duolm_compile(ctypes.byref(tpl), R, _p(hi), _p(ho), _p(fb), _p(fo), _p(ci), _p(co), int(n_items),
+                               int(n_threads), _p(prefix), prefix.size, _p(poff), _p(branch), branch.size)
+    else:
+        hc = np.ascontiguousarray(hist_cached, np.int32)
+        cached = np.zeros(R, np.int32)
+        keep = np.zeros(R, np.int32)
+        rc = lib.duolm_compile_append(ctypes.byref(tpl), R, _p(hi), _p(ho), _p(fb), _p(fo), _p(ci), _p(co),
+                                      int(n_items), int(n_threads), _p(hc), _p(prefix), prefix.size, _p(poff),
+                                      _p(branch), branch.size, _p(cached), _p(keep))
     if rc != 0:
         raise DuolmError(rc, lib.duolm_last_error(None).decode())
-    return prefix[:int(poff[-1])], poff, branch[:int(co[-1]) * b], co, b
+    out = (prefix[:int(poff[-1])], poff, branch[:int(co[-1]) * b], co, b)
+    return out if hist_cached is None else out + (cached, keep)
 
 
 def attention_plan(L, K, cached, branch_len: int, n_kv_heads: int, rows_per_item: int, n_ctas: int):

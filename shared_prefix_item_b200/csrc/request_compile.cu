@@ -43,11 +43,17 @@ bool offsets_ok(const int64_t* off, int64_t n) {
 
 }  // namespace
 
-extern "C" int duolm_compile(const duolm_template* tpl, int n_requests, const int64_t* hist_items,
-                             const int64_t* hist_offsets, const int32_t* feedback, const int64_t* feedback_offsets,
-                             const int64_t* cand_items, const int64_t* cand_offsets, int64_t n_items, int n_threads,
-                             int32_t* prefix_ids, int64_t prefix_capacity, int64_t* prefix_offsets,
-                             int32_t* branch_ids, int64_t branch_capacity) {
+// hist_cached == nullptr: whole prefixes.  Otherwise request r's slot of the
+// prefix KV store holds its instruction and first hist_cached[r] history
+// items (hist_cached[r] < 0: the request does not use the store): only the
+// rest is compiled, and cached_out / keep_out receive the arguments of
+// duolm_prepare_cached.
+static int compile_impl(const duolm_template* tpl, int n_requests, const int64_t* hist_items,
+                        const int64_t* hist_offsets, const int32_t* feedback, const int64_t* feedback_offsets,
+                        const int64_t* cand_items, const int64_t* cand_offsets, int64_t n_items, int n_threads,
+                        const int32_t* hist_cached, int32_t* prefix_ids, int64_t prefix_capacity,
+                        int64_t* prefix_offsets, int32_t* branch_ids, int64_t branch_capacity, int32_t* cached_out,
+                        int32_t* keep_out) {
   g_noctx_err.clear();
   if (!tpl || n_requests < 1 || !hist_offsets || !feedback_offsets || !cand_offsets || !prefix_offsets ||
       n_items < 1 || tpl->vocab < 1 || tpl->m < 1 || tpl->n_instr < 0 || tpl->n_header < 0 ||
@@ -72,15 +78,34 @@ extern "C" int duolm_compile(const duolm_template* tpl, int n_requests, const in
     for (int i = 0; i < t.second; ++i)
       if (t.first[i] < 0 || t.first[i] >= V) return fail(DUOLM_E_ID, "compile: template token %d out of range", t.first[i]);
   if (tpl->marker < 0 || tpl->marker >= V) return fail(DUOLM_E_ID, "compile: marker out of range");
+  if (hist_cached) {
+    if (!cached_out || !keep_out) return fail(DUOLM_E_ARG, "compile: null cached or keep output");
+    for (int r = 0; r < R; ++r)
+      if (hist_cached[r] < -1 || hist_cached[r] > hist_offsets[r + 1] - hist_offsets[r])
+        return fail(DUOLM_E_ARG, "compile: request %d has %lld history items, %d of them cached", r,
+                    (long long)(hist_offsets[r + 1] - hist_offsets[r]), hist_cached[r]);
+  }
+  // first history item each request compiles (the ones before it are in the store)
+  auto first_item = [&](int r) -> int64_t {
+    return hist_offsets[r] + (hist_cached && hist_cached[r] > 0 ? hist_cached[r] : 0);
+  };
+  auto item_len = [&](int64_t h) -> int64_t { return 1 + m + (feedback_offsets[h + 1] - feedback_offsets[h]); };
 
   // lengths and offsets
   const int64_t b = tpl->n_branch_header + m;
   prefix_offsets[0] = 0;
   for (int r = 0; r < R; ++r) {
-    int64_t L = tpl->n_instr + tpl->n_header;
-    for (int64_t h = hist_offsets[r]; h < hist_offsets[r + 1]; ++h)
-      L += 1 + m + (feedback_offsets[h + 1] - feedback_offsets[h]);
+    const int hc = hist_cached ? hist_cached[r] : -1;
+    int64_t stored = hc > 0 ? tpl->n_instr : 0;  // tokens already in the slot
+    for (int64_t h = hist_offsets[r]; h < first_item(r); ++h) stored += item_len(h);
+    int64_t L = (hc > 0 ? 0 : tpl->n_instr) + tpl->n_header;
+    for (int64_t h = first_item(r); h < hist_offsets[r + 1]; ++h) L += item_len(h);
     prefix_offsets[r + 1] = prefix_offsets[r] + L;
+    if (hist_cached) {
+      if (stored > INT32_MAX || L > INT32_MAX) return fail(DUOLM_E_CAPACITY, "compile: request %d too long", r);
+      cached_out[r] = (int32_t)stored;
+      keep_out[r] = hc < 0 ? 0 : (int32_t)(L - tpl->n_header);  // all new history, not the header
+    }
   }
   if (prefix_offsets[R] > prefix_capacity)
     return fail(DUOLM_E_CAPACITY, "compile: %lld prefix tokens, capacity %lld", (long long)prefix_offsets[R],
@@ -102,8 +127,8 @@ extern "C" int duolm_compile(const duolm_template* tpl, int n_requests, const in
   auto work = [&](int w) {
     for (int r = w; r < R; r += T) {
       int32_t* p = prefix_ids + prefix_offsets[r];
-      p = std::copy(tpl->instr, tpl->instr + tpl->n_instr, p);
-      for (int64_t h = hist_offsets[r]; h < hist_offsets[r + 1]; ++h) {
+      if (!(hist_cached && hist_cached[r] > 0)) p = std::copy(tpl->instr, tpl->instr + tpl->n_instr, p);
+      for (int64_t h = first_item(r); h < hist_offsets[r + 1]; ++h) {
         const int64_t it = hist_items[h];
         if ((it < 0 || it >= n_items) && bad[w] < 0) bad[w] = r;
         const int64_t row = std::min<int64_t>(std::max<int64_t>(it, 0), n_items - 1) * m;
@@ -140,4 +165,30 @@ extern "C" int duolm_compile(const duolm_template* tpl, int n_requests, const in
     return fail(DUOLM_E_ID, "compile: request %lld has an item id outside [0, %lld) or a feedback token outside "
                 "the vocabulary", (long long)first_bad, (long long)n_items);
   return DUOLM_OK;
+}
+
+extern "C" int duolm_compile(const duolm_template* tpl, int n_requests, const int64_t* hist_items,
+                             const int64_t* hist_offsets, const int32_t* feedback, const int64_t* feedback_offsets,
+                             const int64_t* cand_items, const int64_t* cand_offsets, int64_t n_items, int n_threads,
+                             int32_t* prefix_ids, int64_t prefix_capacity, int64_t* prefix_offsets,
+                             int32_t* branch_ids, int64_t branch_capacity) {
+  return compile_impl(tpl, n_requests, hist_items, hist_offsets, feedback, feedback_offsets, cand_items, cand_offsets,
+                      n_items, n_threads, nullptr, prefix_ids, prefix_capacity, prefix_offsets, branch_ids,
+                      branch_capacity, nullptr, nullptr);
+}
+
+extern "C" int duolm_compile_append(const duolm_template* tpl, int n_requests, const int64_t* hist_items,
+                                    const int64_t* hist_offsets, const int32_t* feedback,
+                                    const int64_t* feedback_offsets, const int64_t* cand_items,
+                                    const int64_t* cand_offsets, int64_t n_items, int n_threads,
+                                    const int32_t* hist_cached, int32_t* prefix_ids, int64_t prefix_capacity,
+                                    int64_t* prefix_offsets, int32_t* branch_ids, int64_t branch_capacity,
+                                    int32_t* cached_out, int32_t* keep_out) {
+  if (!hist_cached) {
+    g_noctx_err = "compile_append: null hist_cached";
+    return DUOLM_E_ARG;
+  }
+  return compile_impl(tpl, n_requests, hist_items, hist_offsets, feedback, feedback_offsets, cand_items, cand_offsets,
+                      n_items, n_threads, hist_cached, prefix_ids, prefix_capacity, prefix_offsets, branch_ids,
+                      branch_capacity, cached_out, keep_out);
 }

@@ -118,3 +118,53 @@ def test_capacity_is_checked_before_writing(S):
         assert rc == -5
         assert b"capacity" in _lib.lib.duolm_last_error(None)
         assert np.all(prefix == -9) and np.all(branch == -9)
+
+
+def _append_expected(wl, hc):
+    """What the store already holds and what is left, from the generated
+    sequences: with h > 0 items stored the slot holds everything before
+    item h (the instruction and items 0..h-1); h = 0 is an empty slot."""
+    n_header = len(wl.template.header)
+    news, cached, keep = [], [], []
+    for q, r in enumerate(wl.requests):
+        h = hc[q]
+        offs = wl.history_offsets(q) + [r.L - n_header]
+        c = offs[h] if h > 0 else 0
+        news.append(r.prefix_ids[c:])
+        cached.append(c)
+        keep.append(0 if h < 0 else r.L - n_header - c)
+    return np.concatenate(news), cached, keep
+
+
+@pytest.mark.parametrize("recipe", ["c64", "fir"])
+def test_compile_append_matches_the_generated_sequences(S, recipe):
+    wl = W.c64(n_requests=16) if recipe == "c64" else W.fir(m=8, n_requests=16)
+    n_hist = [len(r.history_items) for r in wl.requests]
+    rng = np.random.default_rng(5)
+    hc = [-1, 0] + [int(rng.integers(0, n + 1)) for n in n_hist[2:]]
+    hc[2] = n_hist[2]          # every item stored: only the header is new
+    hc[3] = n_hist[3] - 1      # the next item arrives
+    hist, hoff, fb, foff, cand, coff = wl.records()
+    t = wl.template
+    prefix, poff, branch, coff2, b, cached, keep = S.compile_requests(
+        wl.model.vocab, t.marker, wl.m, t.instr, t.header, t.branch_header[: wl.branch_len - wl.m], hist, hoff, fb,
+        foff, cand, coff, wl.n_items // wl.m, 3, hist_cached=hc)
+    want_ids, want_cached, want_keep = _append_expected(wl, hc)
+    assert np.array_equal(prefix, want_ids)
+    assert list(cached) == want_cached and list(keep) == want_keep
+    assert np.array_equal(branch, wl.packed()[2])
+    # the whole prefix is the stored part followed by the compiled part
+    for q, r in enumerate(wl.requests):
+        assert poff[q + 1] - poff[q] + cached[q] == r.L
+
+
+def test_compile_append_rejects_bad_counts(S):
+    wl = W.c64(n_requests=3)
+    hist, hoff, fb, foff, cand, coff = wl.records()
+    t = wl.template
+    n0 = len(wl.requests[0].history_items)
+    for bad in ([n0 + 1, 0, 0], [-2, 0, 0]):
+        with pytest.raises(S.DuolmError) as e:
+            S.compile_requests(wl.model.vocab, t.marker, 1, t.instr, t.header, t.branch_header[:0], hist, hoff, fb,
+                               foff, cand, coff, wl.n_items, 1, hist_cached=bad)
+        assert e.value.code == -1
