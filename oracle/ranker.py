@@ -27,7 +27,7 @@ prefix once, then every branch, and gives each branch row the prefix keys
 followed by its own branch keys, in the same order as the independent
 sequence, so both layouts reach the same bits through the C core.
 
-Readings where the pages are silent (each listed in the design doc):
+Readings taken where the pages are silent:
 branch token i of a b-token branch sits at position L + i and sees branch
 tokens 0..i; h is the output of the final RMSNorm; there is no score bias;
 RMS in the interface has no epsilon; the interface output is rounded to FP16
