@@ -398,3 +398,63 @@ def test_qk_norm_makes_scores_invariant_to_qk_scale():
     w2 = [a.copy() for a in W.model_weights(TINY)]
     w2[_idx(TINY, "l0.wv")] *= 4.0
     assert not np.allclose(R.score_mis(R.OracleModel(TINY, w2), tab, req), base, atol=1e-3)
+
+
+def _fp16_rne(x) -> float:
+    """Nearest FP16 value of an exact rational (ties to even mantissa)."""
+    from fractions import Fraction
+    x = Fraction(x)
+    if x == 0:
+        return 0.0
+    s, x = (-1 if x < 0 else 1), abs(x)
+    e = max(x.numerator.bit_length() - x.denominator.bit_length() - 1, -14)
+    while Fraction(2) ** e > x and e > -14:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= x:
+        e += 1
+    step = Fraction(2) ** (e - 10)  # 10 fraction bits; subnormal spacing below 2^-14
+    q, r = divmod(x, step)
+    q = int(q)
+    if r * 2 > step or (r * 2 == step and q % 2 == 1):
+        q += 1
+    return s * float(q * step)
+
+
+def test_interface_golden_at_the_pages_rho():
+    """tests/golden/interface_rho.txt: the pages' rho, vectors with rational
+    RMS; the oracle's FP16 table rows equal the exact rational z rounded to
+    nearest even, and RMS(z) = rho before rounding."""
+    import os
+    from fractions import Fraction
+    path = os.path.join(os.path.dirname(__file__), "golden", "interface_rho.txt")
+    rho_s, rows = None, []
+    for line in open(path, encoding="utf-8"):
+        f = line.split()
+        if not f or f[0].startswith("#"):
+            continue
+        if f[0] == "rho":
+            rho_s = f[1]
+        elif f[0] == "gamma":
+            assert float(f[1]) == 0.0
+        elif f[0] == "a":
+            rows.append([Fraction(v) for v in f[1:]])
+    rho = Fraction(rho_s)
+    assert rho == Fraction(280669, 10 ** 7)
+    got = R.interface(np.array([[float(v) for v in a] for a in rows]), 0.0, float(rho))
+    for a, z16 in zip(rows, got):
+        ms = sum(v * v for v in a) / len(a)
+        rms = Fraction(int(round(float(ms) ** 0.5 * 2)), 2)  # the vectors' RMS are halves
+        assert rms * rms == ms
+        z = [rho * v / rms for v in a]
+        assert sum(v * v for v in z) / len(z) == rho * rho  # RMS(z) = rho, exactly
+        assert [float(v) for v in z16] == [_fp16_rne(v) for v in z]
+
+
+def test_fp16_rounding_helper():
+    from fractions import Fraction as F
+    assert _fp16_rne(F(1, 3)) == float(np.float16(1 / 3))
+    assert _fp16_rne(F(-1000, 7)) == float(np.float16(-1000 / 7))
+    assert _fp16_rne(F(1, 2 ** 20)) == 2.0 ** -20              # subnormal, exact
+    assert _fp16_rne(1 + F(1, 2 ** 11)) == 1.0                 # tie to the even mantissa
+    assert _fp16_rne(1 + F(3, 2 ** 11)) == 1 + 2.0 ** -9       # tie to the even mantissa
+    assert _fp16_rne(F(3, 2 ** 25)) == 2.0 ** -23              # subnormal tie: 1.5 ulp -> 2 ulp
