@@ -10,7 +10,11 @@
  *   sections 核心方法 (ranker and score head s = w^T h), 方法步骤详情 steps 3-5
  *   (FP16 item table addressed by virtual id V + i; shared prefix prefilled
  *   once; candidate j sees only the prefix and itself at logical position L_q;
- *   scores in input order; CUDA Graph replay), 研究动机 (s^MIS = s).
+ *   scores in input order; CUDA Graph replay), 研究动机 (s^MIS = s),
+ *   未来方向 (3) (history appended within a session adds only its own K/V:
+ *   the prefix KV store and duolm_prepare_cached).  The request compiler
+ *   (duolm_compile) builds the token sequences of step 3 from item ids and
+ *   feedback on the host.
  *
  * Conventions for every call:
  *   - Return 0 on success, a negative DUOLM_E_* code on failure; the text of
