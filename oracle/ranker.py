@@ -31,7 +31,12 @@ Readings taken where the pages are silent:
 branch token i of a b-token branch sits at position L + i and sees branch
 tokens 0..i; h is the output of the final RMSNorm; there is no score bias;
 RMS in the interface has no epsilon; the interface output is rounded to FP16
-with round-to-nearest-even.
+with round-to-nearest-even; the reference scale rho of the synthetic
+configurations is the mean over embedding rows of each row's RMS.  Every
+arithmetic step runs in fp64 where a plain fp32 ranker would do: fp64 is the
+stricter reading (its own rounding sits far below both tolerances, 1e-4 for
+the fp32 model and 2e-2 std(s) for the bf16-valued one), so a disagreement
+with the GPU path is the GPU path's.
 """
 from __future__ import annotations
 

@@ -87,6 +87,35 @@ def test_interface_rms_closed_form(gamma):
     assert np.all(np.abs(zf - z16) <= np.abs(zf - dn) + 0.0)
 
 
+def test_embedding_rho_is_the_mean_of_row_rms():
+    """rho of the synthetic configurations: the mean over embedding rows of
+    each row's RMS (DuoLM summary page, 前置知识 / 核心方法: z = e^gamma *
+    rho * a / RMS(a), with rho the reference scale of the native embeddings).
+    Rows are chosen with integer RMS, so each reduction someone might write
+    by mistake gives a different number: the RMS of the whole table, the
+    mean of squares, the mean absolute value, an epsilon under the root."""
+    rows = np.array([[4.0, 4.0, 2.0, 0.0],     # RMS 3, mean |x| 2.5
+                     [8.0, -6.0, 0.0, 0.0],    # RMS 5, mean |x| 3.5
+                     [0.5, -0.5, 0.5, 0.5]])   # RMS 0.5
+    for scale in (1.0, 2.0 ** -6):             # 2^-6: the N(0, 0.02) range, still exact
+        e = rows * scale
+        want = (3.0 + 5.0 + 0.5) / 3.0 * scale
+        got = R.embedding_rho(e.astype(np.float32))
+        assert got == pytest.approx(want, rel=1e-15, abs=0)
+        assert abs(float(np.sqrt(np.mean(e * e))) - want) > 0.1 * want     # RMS of the whole table
+        assert abs(float(np.mean(e * e)) - want) > 0.1 * want              # mean of squares
+        assert abs(float(np.mean(np.abs(e))) - want) > 0.1 * want          # mean |x|
+    # an epsilon under the root would move the result: no epsilon here
+    tiny = np.full((2, 4), 2.0 ** -20, np.float32)
+    assert R.embedding_rho(tiny) == 2.0 ** -20
+    # rows are independent of their order; scaling one row by s moves rho by
+    # (s - 1) RMS(row) / n_rows
+    assert R.embedding_rho(rows[::-1].astype(np.float32)) == pytest.approx(8.5 / 3.0, rel=1e-15)
+    r2 = rows.copy()
+    r2[1] *= 4.0
+    assert R.embedding_rho(r2.astype(np.float32)) == pytest.approx((3.0 + 20.0 + 0.5) / 3.0, rel=1e-15)
+
+
 def test_interface_scale_invariance():
     # RMS normalisation makes z independent of the scale of a.
     a = W.item_vectors(16, 128).astype(np.float64)
