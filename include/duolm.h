@@ -206,7 +206,15 @@ int duolm_sync(duolm_ctx *ctx);
 
 /*
  * One whole call: prepare + execute + copy the scores to host memory
- * (scores_out: host float [cand_offsets[n_requests]]) + synchronise.
+ * (scores_out: host float [cand_offsets[n_requests]]) + synchronise.  This is
+ * the request-level operation of the DuoLM summary page (paper.rainbus.top),
+ * 方法步骤详情 step 4: the K candidates of a request are packed behind its
+ * shared prefix, the prefix is prefilled once, each candidate sees only the
+ * prefix and its own branch at the unified logical positions, and the K
+ * scores s = w^T h come back in input order.  Arguments as duolm_prepare;
+ * scores_out is caller-owned host memory, written before the call returns.
+ * Errors as duolm_prepare and duolm_execute, plus DUOLM_E_DEVICE when a
+ * kernel raised the device error flag.
  */
 int duolm_score(duolm_ctx *ctx, int n_requests, const int32_t *prefix_ids,
                 const int64_t *prefix_offsets, const int32_t *branch_ids,
@@ -257,8 +265,8 @@ typedef struct {
  *   cand_items [cand_offsets[n_requests]], cand_offsets [n_requests + 1]
  *     (every request has at least one candidate);
  *   n_items: table items (ids must be < n_items); n_threads > 0: that many
- *     worker threads (at most n_requests), <= 0: one per 256K output tokens,
- *     at most the host's hardware threads.
+ *     worker threads (at most n_requests and the host's hardware threads),
+ *     <= 0: one per 256K output tokens, at most the host's hardware threads.
  * Output (caller-owned host arrays): prefix_ids [prefix_capacity] and
  * prefix_offsets [n_requests + 1]; branch_ids [branch_capacity], candidate
  * c's branch at c * branch_len (the candidate offsets are cand_offsets).
@@ -285,7 +293,8 @@ int duolm_compile(const duolm_template *tpl, int n_requests, const int64_t *hist
  * cached_out[r] receives the tokens the slot holds (the instruction and the
  * first h items; 0 for h = 0), keep_out[r] the new prefix tokens to append
  * (everything but the header), both ready for duolm_prepare_cached.
- * Errors as duolm_compile; DUOLM_E_ARG also for h outside -1..items.
+ * Errors as duolm_compile (on DUOLM_E_CAPACITY cached_out and keep_out are
+ * not written either); DUOLM_E_ARG also for h outside -1..items.
  */
 int duolm_compile_append(const duolm_template *tpl, int n_requests, const int64_t *hist_items,
                          const int64_t *hist_offsets, const int32_t *feedback,
@@ -340,16 +349,20 @@ int duolm_gather(duolm_ctx *ctx, const int32_t *ids, int64_t n, float *x, uint16
  *   rho_out: device pointer to one double; written by the call.
  *   cuda_stream: the cudaStream_t to launch on (NULL: the default stream).
  * The call only enqueues work on the stream of the current device and
- * returns; rho_out is valid once that stream has reached it.  The first call
- * on each device looks up the scratch array's device address (with that
- * device current) and caches it; make that first call before any stream
- * capture.  Every element of the scratch a call reads is first written by
- * the same call, so nothing needs clearing, but all calls in the process
- * share the one array: calls whose work overlaps on the GPU (different
- * streams, no ordering between them) race and may return wrong results.
- * Returns 0; DUOLM_E_ARG for a null pointer, d < 1 or a bad dtype;
- * DUOLM_E_CAPACITY when vocab is < 1 or above DUOLM_RHO_STATIC_MAX_ROWS;
- * DUOLM_E_CUDA when the address lookup or a launch fails.
+ * returns; rho_out is valid once that stream has reached it.  Outside stream
+ * capture every call looks up the scratch array's device address with the
+ * device current (so a reset device or a new context is followed); while the
+ * stream is being captured the address from the last call outside capture
+ * on that device is used, so make the first call on each device before any
+ * stream capture (DUOLM_E_STATE otherwise).  Every element of the scratch a
+ * call reads is first written by the same call, so nothing needs clearing,
+ * but all calls in the process share the one array: calls whose work
+ * overlaps on the GPU (different streams, no ordering between them) race and
+ * may return wrong results.  A CUDA error left pending by earlier work is
+ * reported (DUOLM_E_CUDA) before anything is enqueued.  Returns 0;
+ * DUOLM_E_ARG for a null pointer, d < 1 or a bad dtype; DUOLM_E_CAPACITY when
+ * vocab is < 1 or above DUOLM_RHO_STATIC_MAX_ROWS; DUOLM_E_CUDA when the
+ * address lookup or a launch fails; the reason in duolm_last_error(NULL).
  */
 int duolm_embedding_rho_static(const void *embed, int dtype, int64_t vocab, int d, double *rho_out,
                                void *cuda_stream);

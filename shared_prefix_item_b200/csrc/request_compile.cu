@@ -93,6 +93,8 @@ static int compile_impl(const duolm_template* tpl, int n_requests, const int64_t
 
   // lengths and offsets
   const int64_t b = tpl->n_branch_header + m;
+  // cached / keep are written only once the capacities are known to hold
+  std::vector<int32_t> cached_v(hist_cached ? R : 0), keep_v(hist_cached ? R : 0);
   prefix_offsets[0] = 0;
   for (int r = 0; r < R; ++r) {
     const int hc = hist_cached ? hist_cached[r] : -1;
@@ -103,8 +105,8 @@ static int compile_impl(const duolm_template* tpl, int n_requests, const int64_t
     prefix_offsets[r + 1] = prefix_offsets[r] + L;
     if (hist_cached) {
       if (stored > INT32_MAX || L > INT32_MAX) return fail(DUOLM_E_CAPACITY, "compile: request %d too long", r);
-      cached_out[r] = (int32_t)stored;
-      keep_out[r] = hc < 0 ? 0 : (int32_t)(L - tpl->n_header);  // all new history, not the header
+      cached_v[r] = (int32_t)stored;
+      keep_v[r] = hc < 0 ? 0 : (int32_t)(L - tpl->n_header);  // all new history, not the header
     }
   }
   if (prefix_offsets[R] > prefix_capacity)
@@ -114,14 +116,17 @@ static int compile_impl(const duolm_template* tpl, int n_requests, const int64_t
     return fail(DUOLM_E_CAPACITY, "compile: %lld branch tokens, capacity %lld", (long long)(C * b),
                 (long long)branch_capacity);
   if ((prefix_offsets[R] && !prefix_ids) || !branch_ids) return fail(DUOLM_E_ARG, "compile: null output array");
+  if (hist_cached) {
+    std::copy(cached_v.begin(), cached_v.end(), cached_out);
+    std::copy(keep_v.begin(), keep_v.end(), keep_out);
+  }
 
   // every request's slice; a worker records the first bad id of its range
   // Starting a thread costs tens of microseconds, about what one thread
   // needs to write 64K tokens: by default one worker per 256K tokens.
   const int64_t tokens = prefix_offsets[R] + C * b;
-  int T = n_threads;
-  if (T <= 0)
-    T = (int)std::min<int64_t>(std::max(1u, std::thread::hardware_concurrency()), 1 + tokens / (1 << 18));
+  const int hw = (int)std::max(1u, std::thread::hardware_concurrency());
+  int T = n_threads > 0 ? std::min(n_threads, hw) : (int)std::min<int64_t>(hw, 1 + tokens / (1 << 18));
   T = std::min(T, R);
   std::vector<int64_t> bad(T, -1);  // request index of a bad id, per worker
   auto work = [&](int w) {

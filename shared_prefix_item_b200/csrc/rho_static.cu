@@ -1,10 +1,18 @@
 // duolm_embedding_rho_static: the embedding's reference scale rho computed
 // with a scratch array built into the library instead of allocated memory,
-// for callers that cannot allocate device memory (see include/duolm.h).
+// for callers that cannot allocate device memory (see include/duolm.h).  The
+// arithmetic is the context's own (duolm::embed_rho: per-row RMS in fp64,
+// then their mean); only where the per-row values live differs.
+#include <cstdio>
 #include <mutex>
+#include <string>
 
 #include "common.cuh"
 #include "duolm.h"
+#include "kernels.cuh"
+
+// reason of the calling thread's last failed context-free call (runtime.cu)
+extern thread_local std::string g_noctx_err;
 
 namespace {
 
@@ -16,81 +24,62 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) double g_rho_rows[kMaxRows];
 
 std::mutex g_mu;
-double* g_rows_addr[kMaxDevices] = {};  // device address of g_rho_rows, per device
+double* g_rows_addr[kMaxDevices] = {};  // last looked-up address of g_rho_rows, per device
 
-// RMS of each embedding row in fp64, one block per row (fixed-order reduction).
-__global__ void rho_rows_kernel(const void* __restrict__ embed, bool bf16, int64_t vocab, int d,
-                                double* __restrict__ rows) {
-  __shared__ double red[256];
-  for (int64_t r = blockIdx.x; r < vocab; r += gridDim.x) {
-    double ss = 0.0;
-    for (int i = threadIdx.x; i < d; i += blockDim.x) {
-      double v;
-      if (bf16) {
-        const uint16_t u = reinterpret_cast<const uint16_t*>(embed)[r * d + i];
-        v = (double)__uint_as_float((uint32_t)u << 16);
-      } else {
-        v = (double)reinterpret_cast<const float*>(embed)[r * d + i];
-      }
-      ss += v * v;
-    }
-    red[threadIdx.x] = ss;
-    __syncthreads();
-    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
-      if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
-      __syncthreads();
-    }
-    if (threadIdx.x == 0) rows[r] = sqrt(red[0] / (double)d);
-    __syncthreads();
-  }
+int fail_cuda(const char* what, cudaError_t e) {
+  char buf[256];
+  std::snprintf(buf, sizeof buf, "embedding_rho_static: %s: %s", what, cudaGetErrorString(e));
+  g_noctx_err = buf;
+  return DUOLM_E_CUDA;
 }
 
-// Mean of the per-row values, one block, fixed-order reduction.
-__global__ void rho_mean_kernel(const double* __restrict__ rows, int64_t vocab, double* __restrict__ out) {
-  __shared__ double red[1024];
-  double s = 0.0;
-  for (int64_t i = threadIdx.x; i < vocab; i += blockDim.x) s += rows[i];
-  red[threadIdx.x] = s;
-  __syncthreads();
-  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
-    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) *out = red[0] / (double)vocab;
-}
-
-// Device address of the scratch array on the current device, looked up once
-// per device (host code cannot use the array's name as a device pointer).
-cudaError_t rows_address(double** out) {
+// Device address of the scratch array on the current device.  Host code
+// cannot use the array's name as a device pointer, so the address is looked
+// up with the device current.  Outside stream capture it is looked up on
+// every call (a reset device or another context may have moved the module);
+// while the stream is being captured the address of the last call outside
+// capture on this device is used, so one such call must come first.
+int rows_address(cudaStream_t s, double** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (e != cudaSuccess) return fail_cuda("cudaGetDevice", e);
+  if (dev < 0 || dev >= kMaxDevices) return fail_cuda("device index", cudaErrorInvalidDevice);
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if ((e = cudaStreamIsCapturing(s, &cap)) != cudaSuccess) return fail_cuda("cudaStreamIsCapturing", e);
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_rows_addr[dev]) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_rho_rows);
-    if (e != cudaSuccess) return e;
+    if ((e = cudaGetSymbolAddress(&p, g_rho_rows)) != cudaSuccess) return fail_cuda("cudaGetSymbolAddress", e);
     g_rows_addr[dev] = static_cast<double*>(p);
+  } else if (!g_rows_addr[dev]) {
+    g_noctx_err = "embedding_rho_static: first call on this device made during stream capture";
+    return DUOLM_E_STATE;
   }
   *out = g_rows_addr[dev];
-  return cudaSuccess;
+  return 0;
 }
 
 }  // namespace
 
 extern "C" int duolm_embedding_rho_static(const void* embed, int dtype, int64_t vocab, int d, double* rho_out,
                                           void* cuda_stream) {
-  if (!embed || !rho_out || d < 1 || (dtype != DUOLM_DTYPE_BF16 && dtype != DUOLM_DTYPE_FP32))
+  g_noctx_err.clear();
+  if (!embed || !rho_out || d < 1 || (dtype != DUOLM_DTYPE_BF16 && dtype != DUOLM_DTYPE_FP32)) {
+    g_noctx_err = "embedding_rho_static: null pointer, d < 1 or unknown dtype";
     return DUOLM_E_ARG;
-  if (vocab < 1 || vocab > kMaxRows) return DUOLM_E_CAPACITY;
-  double* rows = nullptr;
-  if (rows_address(&rows) != cudaSuccess) return DUOLM_E_CUDA;
+  }
+  if (vocab < 1 || vocab > kMaxRows) {
+    g_noctx_err = "embedding_rho_static: vocab outside [1, DUOLM_RHO_STATIC_MAX_ROWS]";
+    return DUOLM_E_CAPACITY;
+  }
+  // an error left by earlier work is reported now, before anything is
+  // enqueued, so that a failed call has launched nothing
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail_cuda("error pending before the call", e);
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
-  const int grid = (int)(vocab < 148 * 16 ? vocab : 148 * 16);
-  rho_rows_kernel<<<grid, 256, 0, s>>>(embed, dtype == DUOLM_DTYPE_BF16, vocab, d, rows);
-  if (cudaGetLastError() != cudaSuccess) return DUOLM_E_CUDA;
-  rho_mean_kernel<<<1, 1024, 0, s>>>(rows, vocab, rho_out);
-  if (cudaGetLastError() != cudaSuccess) return DUOLM_E_CUDA;
+  double* rows = nullptr;
+  if (const int rc = rows_address(s, &rows)) return rc;
+  if ((e = duolm::embed_rho(embed, dtype == DUOLM_DTYPE_BF16, vocab, d, rows, rho_out, s)) != cudaSuccess)
+    return fail_cuda("launch", e);
   return 0;
 }

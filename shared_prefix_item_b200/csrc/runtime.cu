@@ -936,10 +936,14 @@ int duolm_execute(duolm_ctx* ctx) {
   if (!ctx->prepared) return fail(ctx, DUOLM_E_STATE, "execute: nothing prepared");
   CK(cudaSetDevice(ctx->device));
   // the slots this batch appends to hold its rows once the launches below
-  // have run (work on the same stream sees them)
-  for (const auto& u : ctx->slot_update) ctx->slot_len[u.first] = u.second;
+  // have run (work on the same stream sees them); the lengths change only
+  // after the whole pass was enqueued, so a failed call leaves them as they were
+  auto commit_slots = [ctx]() {
+    for (const auto& u : ctx->slot_update) ctx->slot_len[u.first] = u.second;
+  };
   if (!ctx->use_graph) {
     CK(launch_forward(ctx, ctx->desc.n_layers, true, &ctx->launches));
+    commit_slots();
     return 0;
   }
   if (!ctx->graph_valid) {
@@ -960,6 +964,7 @@ int duolm_execute(duolm_ctx* ctx) {
     ctx->launches = n;
   }
   CK(cudaGraphLaunch(ctx->gexec, ctx->stream));
+  commit_slots();
   return 0;
 }
 

@@ -118,6 +118,29 @@ def test_capacity_is_checked_before_writing(S):
         assert rc == -5
         assert b"capacity" in _lib.lib.duolm_last_error(None)
         assert np.all(prefix == -9) and np.all(branch == -9)
+        # the append form leaves its cached / keep outputs untouched as well
+        hc = np.zeros(3, np.int32)
+        cached = np.full(3, -9, np.int32)
+        keep = np.full(3, -9, np.int32)
+        rc = _lib.lib.duolm_compile_append(ctypes.byref(tpl), 3, _lib._p(hist), _lib._p(hoff), _lib._p(fb),
+                                           _lib._p(foff), _lib._p(cand), _lib._p(coff), wl.n_items, 2, _lib._p(hc),
+                                           _lib._p(prefix), pcap, _lib._p(poff), _lib._p(branch), bcap,
+                                           _lib._p(cached), _lib._p(keep))
+        assert rc == -5
+        assert np.all(cached == -9) and np.all(keep == -9)
+        assert np.all(prefix == -9) and np.all(branch == -9)
+
+
+def test_thread_count_above_the_host_threads_is_capped(S):
+    # a caller asking for far more workers than the host has gets the same
+    # output (the count is capped at the hardware threads, not honoured)
+    wl = W.c64(n_requests=64)
+    hist, hoff, fb, foff, cand, coff = wl.records()
+    t = wl.template
+    out = S.compile_requests(wl.model.vocab, t.marker, 1, t.instr, t.header, t.branch_header[:0], hist, hoff, fb,
+                             foff, cand, coff, wl.n_items, 100000)
+    want = wl.packed()
+    assert np.array_equal(out[0], want[0]) and np.array_equal(out[2], want[2])
 
 
 def _append_expected(wl, hc):
