@@ -568,26 +568,57 @@ def run_latency(args, rank: int, world: int, local_rank: int) -> None:
     rk.close()
 
 
-def run_ours(args, rank: int, world: int, local_rank: int) -> None:
-    import torch
+class CudaDevice:
+    """What run_ours needs from this rank's GPU: the library's context on
+    it, the stream the library launches on (the CUDA events are recorded on
+    it), a device synchronise, the process-group backend and the clock
+    sampler.  The multi-rank CPU test passes a stand-in with the same
+    methods, so that the control flow under N ranks runs without a GPU."""
+    dist_backend = "nccl"
+    tensor_device = "cuda"
 
+    def __init__(self, local_rank: int):
+        import torch
+        torch.cuda.set_device(local_rank)
+        self.torch = torch
+        self.local_rank = local_rank
+        self.stream = torch.cuda.Stream()
+        torch.cuda.set_stream(self.stream)
+
+    def ranker(self, shape, weights):
+        import shared_prefix_item_b200 as S
+        return S.Ranker(shape, weights, device=self.local_rank, stream=self.stream.cuda_stream)
+
+    def events(self):
+        E = self.torch.cuda.Event
+        return E(enable_timing=True), E(enable_timing=True)
+
+    def synchronize(self):
+        self.torch.cuda.synchronize()
+
+    def clock_sampler(self):
+        props = self.torch.cuda.get_device_properties(self.local_rank)
+        gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(self.local_rank)
+        return ClockSampler(gpu_id)
+
+
+def run_ours(args, rank: int, world: int, local_rank: int, dev=None) -> None:
     import shared_prefix_item_b200 as S
 
-    torch.cuda.set_device(local_rank)
+    dev = dev or CudaDevice(local_rank)
     dist = None
     if world > 1:
         import datetime
 
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        dist.init_process_group(dev.dist_backend, timeout=datetime.timedelta(seconds=300))
 
     wl = workload(args.config, rank)
     shape = wl.model
     mode = S.MODE_INDEPENDENT if args.mode == "independent" else S.MODE_MIS
-    # the library launches on this stream; the CUDA events below are recorded on it
-    stream = torch.cuda.Stream()
-    torch.cuda.set_stream(stream)
-    rk = S.Ranker(shape, W.model_weights(shape), device=local_rank, stream=stream.cuda_stream)
+    # the library launches on dev.stream; the events below are recorded on it
+    stream = dev.stream
+    rk = dev.ranker(shape, W.model_weights(shape))
     table_note = load_table(rk, wl.n_items, shape.d)
     rk.set_graph(not args.no_graph)
     p, po, b, co = wl.packed()
@@ -630,12 +661,10 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     def barrier():
         if dist:
             dist.barrier()
-        torch.cuda.synchronize()
+        dev.synchronize()
 
-    props = torch.cuda.get_device_properties(local_rank)
-    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local_rank)
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(gpu_id) as clk:
+    start, end = dev.events()
+    with dev.clock_sampler() as clk:
         barrier()
         start.record(stream)
         for _ in range(args.steps):
@@ -644,7 +673,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         barrier()
     rk.sync()
     ms = start.elapsed_time(end) / args.steps
-    ms_max, n_total = combine_ranks(dist, ms, n_cand, "cuda")
+    ms_max, n_total = combine_ranks(dist, ms, n_cand, dev.tensor_device)
     value = n_total / (ms_max / 1e3)
     launches = rk.launches_per_execute()
 
@@ -659,7 +688,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     end.record(stream)
     barrier()
     e2e_ms = start.elapsed_time(end) / args.steps
-    e2e_max, _ = combine_ranks(dist, e2e_ms, n_cand, "cuda")
+    e2e_max, _ = combine_ranks(dist, e2e_ms, n_cand, dev.tensor_device)
     e2e_value = n_total / (e2e_max / 1e3)
 
     # per-kernel-class device time (eager launches with an event after each)
@@ -695,7 +724,21 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
              "traffic": None if reuse else captured_traffic(k, args.config)}
         r["frac"] = r["achieved"] / r["peak"]
         if k == "attention":
-            r["hbm_gbs_algorithmic"] = attention_bytes(shape, T) / (ms_k / 1e3) / 1e9
+            # the kernel's floor is the slower of its FLOPs at the tensor peak
+            # and its bytes (q, k, v read, o written) at the HBM peak; report
+            # against whichever is larger
+            by = attention_bytes(shape, T)
+            t_s = ms_k / 1e3
+            t_flop = fl / (pk["tc_sustained"] * 1e12)
+            t_byte = by / (pk["hbm"] * 1e9)
+            r["hbm_gbs_algorithmic"] = by / t_s / 1e9
+            r["bytes_per_launch"] = by / n_k
+            r["floor_us_per_launch"] = max(t_flop, t_byte) * 1e6 / n_k
+            r["tensor_frac"] = r["frac"]
+            if t_byte > t_flop:
+                r.update({"bound": "hbm", "achieved": by / t_s / 1e9, "peak": pk["hbm"], "unit": "GB/s",
+                          "peak_note": f"{pk['src']} HBM copy bandwidth (the byte floor is above the FLOP floor)"})
+            r["frac"] = max(t_flop, t_byte) / t_s
             if reuse:
                 r["note"] = "K/V read from the store not counted in the algorithmic bytes"
         roofs[k] = r
@@ -741,6 +784,20 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         dist.destroy_process_group()
 
 
+def relaunch(n: int, argv=None) -> int:
+    """`--gpus N` without a launcher: run this same command as N ranks, one
+    process per GPU, through torch's own launcher on this node (rendezvous
+    on 127.0.0.1); returns the launcher's exit status."""
+    import socket
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__),
+           *(sys.argv[1:] if argv is None else argv)]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -762,6 +819,10 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        sys.exit(relaunch(args.gpus))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE is {world}: launch one process per GPU")
     if args.impl == "reference":
         run_reference(args, rank, world)
     elif args.config == "gather":
