@@ -82,3 +82,19 @@ def split_scores(wl: W.Workload, flat: np.ndarray):
         out.append(flat[o:o + r.K])
         o += r.K
     return out
+
+
+def single_candidate_tolerance(shape: W.ModelShape, om, otab, req: W.Request, n_items: int, seed: int = 7) -> float:
+    """Tolerance for a request with K = 1, where the std over its own scores
+    is 0: 2e-2 times the std of the oracle's scores of 16 seeded random
+    candidates on the same prefix (branches of the same length, the last
+    token a table row, the others vocabulary tokens)."""
+    if shape.dtype == "fp32":
+        return TOL_FP32
+    rng = np.random.default_rng(seed)
+    b = req.branch_ids.shape[1]
+    br = np.empty((16, b), np.int32)
+    br[:, :-1] = rng.integers(0, shape.vocab, size=(16, b - 1))
+    br[:, -1] = shape.vocab + rng.choice(n_items, size=16, replace=False)
+    ref = R.score_mis(om, otab, W.Request(req.prefix_ids, br))
+    return TOL_BF16_REL_STD * float(np.std(ref))

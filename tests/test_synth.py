@@ -16,3 +16,9 @@ def test_zipf_lookup_stream_is_seeded_and_zipf_shaped():
     for k in (1, 2, 10):
         p = k ** -1.1 / H
         assert abs(counts[k - 1] / n - p) < 5 * np.sqrt(p / n), k
+
+
+def test_item_vector_rows_do_not_depend_on_the_draw_length():
+    # the GPU parity tests draw only the rows up to the largest one a request
+    # touches: the stream is counter-based, so those rows equal the full draw's
+    assert np.array_equal(W.item_vectors(300, 64), W.item_vectors(1000, 64)[:300])
