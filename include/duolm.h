@@ -223,6 +223,13 @@ int duolm_score(duolm_ctx *ctx, int n_requests, const int32_t *prefix_ids,
 /* Launch through a captured CUDA graph (1, default) or kernel by kernel (0). */
 int duolm_set_graph(duolm_ctx *ctx, int enabled);
 
+/* Programmatic dependent launch between the pass's kernels (1, default):
+ * each kernel after the first may be scheduled while its predecessor
+ * finishes and runs its prologue (barrier set-up, tensor-memory allocation)
+ * before waiting for the predecessor's results; 0 launches every kernel
+ * after its predecessor has completed.  Results are the same either way. */
+int duolm_set_pdl(duolm_ctx *ctx, int enabled);
+
 /* Number of kernel launches one duolm_execute issues for the prepared batch
  * (graph nodes when the graph is used). */
 int64_t duolm_launches_per_execute(const duolm_ctx *ctx);
@@ -410,7 +417,8 @@ int64_t duolm_plan_bytes(const duolm_ctx *ctx);
  * One projection of layer `layer` through the tensor-core GEMM alone
  * (BF16 models only): out = a * W^T with W = wqkv (which 0, [qd+2kd][d]),
  * wo (1, [d][qd]), gate/up (2, [2*ffn][d], rows in 128-row blocks alternating
- * gate and up) or w_down (3, [d][ffn]).  a: host uint16 fp16 bit patterns
+ * gate and up) or w_down (3, [d][ffn]); which + 4 runs the same product
+ * with the 64-column tiles small batches use.  a: host uint16 fp16 bit patterns
  * [n_tokens][K] where n_tokens is the prepared batch's token count; out: host
  * float [n_tokens][N].  Overwrites the batch's activations.  Synchronous.
  */

@@ -62,6 +62,7 @@ def _load():
         "duolm_sync": (I, [VP]),
         "duolm_score": (I, [VP, I, VP, VP, VP, VP, I, I, VP]),
         "duolm_set_graph": (I, [VP, I]),
+        "duolm_set_pdl": (I, [VP, I]),
         "duolm_launches_per_execute": (I64, [VP]),
         "duolm_last_error": (ctypes.c_char_p, [VP]),
         "duolm_destroy": (None, [VP]),
@@ -297,6 +298,10 @@ class Ranker:
 
     def set_graph(self, enabled: bool):
         self._check(lib.duolm_set_graph(self.ctx, 1 if enabled else 0))
+
+    def set_pdl(self, enabled: bool):
+        """Programmatic dependent launch between the pass's kernels (default on)."""
+        self._check(lib.duolm_set_pdl(self.ctx, 1 if enabled else 0))
 
     def launches_per_execute(self) -> int:
         return int(lib.duolm_launches_per_execute(self.ctx))

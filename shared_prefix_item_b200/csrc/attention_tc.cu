@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](int i) { return smem_u32(bars + i); };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + B_COUNT);
 
-  if (*reinterpret_cast<volatile const uint32_t*>(&st->flags) & ERR_WAIT_TIMEOUT) return;
+  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = plan->branch_len;
   constexpr int R = kSub / G;
@@ -197,11 +197,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  // everything below reads what the previous kernels wrote; a bounded wait
+  // that already gave up in an earlier launch makes the CTA skip its work
+  pdl_wait();
+  const bool skip = (*reinterpret_cast<volatile const uint32_t*>(&st->flags) & ERR_WAIT_TIMEOUT) != 0;
 
   // Every role walks the same items and tiles, so the running counts below
   // (K/V tiles, and per sub-tile its items and tiles) agree across roles and
   // give each barrier's phase.
-  if (warp < 8) {
+  if (skip) {
+    // nothing to do: straight to the teardown
+  } else if (warp < 8) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegSoftmax));
     // ---- softmax of sub-tile X: thread = slot row r = TMEM lane
     const int X = warp >> 2;
@@ -482,26 +488,23 @@ cudaError_t attention_tc_setup() {
 cudaError_t attention_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tks,
                          const CUtensorMap& tvs, const PlanHdr* plan, const int2* reqx, int64_t kv_rows,
                          int64_t store_rows, int n_q_heads, int n_kv_heads, float scale, __half* o, DevStatus* st,
-                         int grid, cudaStream_t s) {
+                         int grid, cudaStream_t s, bool pdl) {
   const int G = n_q_heads / n_kv_heads;
   const float sl2 = scale * 1.4426950408889634f;  // softmax in base 2
+  auto run = [&](auto kernel) {
+    return launch_ex(kernel, dim3(grid), dim3(kThreads), kSmem, s, pdl, tq, tk, tv, tks, tvs, plan, reqx, kv_rows,
+                     store_rows, n_q_heads, sl2, o, st);
+  };
   switch (G) {
     case 1:
-      attention_tc_kernel<1><<<grid, kThreads, kSmem, s>>>(tq, tk, tv, tks, tvs, plan, reqx, kv_rows, store_rows,
-                                                           n_q_heads, sl2, o, st);
-      break;
+      return run(attention_tc_kernel<1>);
     case 2:
-      attention_tc_kernel<2><<<grid, kThreads, kSmem, s>>>(tq, tk, tv, tks, tvs, plan, reqx, kv_rows, store_rows,
-                                                           n_q_heads, sl2, o, st);
-      break;
+      return run(attention_tc_kernel<2>);
     case 4:
-      attention_tc_kernel<4><<<grid, kThreads, kSmem, s>>>(tq, tk, tv, tks, tvs, plan, reqx, kv_rows, store_rows,
-                                                           n_q_heads, sl2, o, st);
-      break;
+      return run(attention_tc_kernel<4>);
     default:
       return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 }  // namespace duolm

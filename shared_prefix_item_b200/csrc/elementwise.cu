@@ -135,6 +135,8 @@ __global__ void __launch_bounds__(kRowThreads)
                       const __half* __restrict__ table, int64_t n_table, int vocab, int d,
                       const float* __restrict__ gain, float* __restrict__ x, __half* __restrict__ xg,
                       float* __restrict__ ssp, int n_slots, DevStatus* st) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int T = plan->n_tokens;
   const int* ids = plan_array<int32_t>(plan, plan->off_ids);
   const int lane = threadIdx.x & 31;
@@ -177,14 +179,15 @@ __global__ void __launch_bounds__(kRowThreads)
 
 cudaError_t embed_gain(const PlanHdr* plan, const void* embed, const __half* table, int64_t n_table, int vocab, int d,
                        const float* gain, float* x, __half* xg, float* ssp, int n_slots, DevStatus* st, int max_rows,
-                       cudaStream_t s) {
+                       cudaStream_t s, bool pdl) {
   const int g = std::max(1, std::min((max_rows + 7) / 8, kMaxRowBlocks));
   if (d % 8 || n_slots > 32 || n_slots % 4) return cudaErrorInvalidValue;
   switch ((d + 255) / 256) {
 #define DUOLM_EG_CASE(n)                                                                                            \
   case n:                                                                                                           \
-    embed_gain_kernel<n><<<g, kRowThreads, 0, s>>>(plan, embed, table, n_table, vocab, d, gain, x, xg, ssp, n_slots, \
-                                                   st);                                                             \
+    if (cudaError_t e_ = launch_ex(embed_gain_kernel<n>, dim3(g), dim3(kRowThreads), 0, s, pdl, plan, embed, table,   \
+                                   n_table, vocab, d, gain, x, xg, ssp, n_slots, st))                                 \
+      return e_;                                                                                                    \
     break;
     DUOLM_EG_CASE(1) DUOLM_EG_CASE(2) DUOLM_EG_CASE(3) DUOLM_EG_CASE(4) DUOLM_EG_CASE(8)
 #undef DUOLM_EG_CASE
@@ -287,6 +290,7 @@ __global__ void __launch_bounds__(kRowThreads)
     score_head_kernel(const PlanHdr* __restrict__ plan, const float* __restrict__ x, int d,
                       const float* __restrict__ gain, const float* __restrict__ w, float eps,
                       float* __restrict__ scores) {
+  pdl_wait();
   const int n = plan->n_cand;
   const int* rows = plan_array<int32_t>(plan, plan->off_cand);
   const int lane = threadIdx.x & 31;
@@ -305,9 +309,9 @@ __global__ void __launch_bounds__(kRowThreads)
 }
 
 cudaError_t score_head(const PlanHdr* plan, const float* x, int d, const float* gain, const float* w, float eps,
-                       float* scores, int max_cand, cudaStream_t s) {
-  score_head_kernel<<<row_blocks(max_cand), kRowThreads, 0, s>>>(plan, x, d, gain, w, eps, scores);
-  return cudaGetLastError();
+                       float* scores, int max_cand, cudaStream_t s, bool pdl) {
+  return launch_ex(score_head_kernel, dim3(row_blocks(max_cand)), dim3(kRowThreads), 0, s, pdl, plan, x, d, gain, w,
+                   eps, scores);
 }
 
 // ---------------------------------------------------------------------------

@@ -37,12 +37,16 @@ constexpr int kBK = 64;  // one 128-byte swizzle row of fp16
 // an A row block and it is read from DRAM once.
 // An epilogue may ask for shared-memory scratch per epilogue warp (then the
 // ring is shallower, so the CTA stays near 197 KB of shared memory).
+// Narrower tiles (BN 64 or 128, one epilogue group) serve small batches,
+// where 256-wide tiles leave most CTA pairs without work; their smaller
+// stages let the ring hold more k-blocks in the same shared memory.
 template <int BN, class Epi>
 struct TcCfg {
-  static constexpr int STAGES = Epi::STAGES;
   static constexpr int A_BYTES = kBM * kBK * 2;        // this CTA's 128 rows of A
   static constexpr int B_BYTES = (BN / 2) * kBK * 2;   // this CTA's half of the B tile
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES_FIT = Epi::STAGES * (kBM * kBK * 2 + 128 * kBK * 2) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT < 8 ? STAGES_FIT : 8;
   static constexpr int EPI_OFF = STAGES * STAGE_BYTES;
   static constexpr int BAR_OFF = EPI_OFF + 4 * Epi::EG * Epi::SCRATCH_PER_WARP;
   static constexpr int SMEM = BAR_OFF + 256 + 1024;    // barriers + alignment slack
@@ -113,9 +117,10 @@ __device__ __forceinline__ void warp_store_rows_128B(uint32_t* buf, const uint32
   warp_flush_rows_128B(buf, dst);
 }
 
-struct EpiResid {
+template <int EG_>
+struct EpiResidT {
   EpiResidArgs a;
-  static constexpr int EG = 2;
+  static constexpr int EG = EG_;
   static constexpr int STAGES = 5;
   static constexpr int kPad = kScratchPad;
   static constexpr int SCRATCH_PER_WARP = kScratchPerWarp;
@@ -253,9 +258,10 @@ struct EpiSwiglu {
 // Per 128-column head of the fused Q|K|V output: q and k get RMSNorm over the
 // head (QK-norm) and rotate-half RoPE at the token's logical position; v is
 // copied.  q goes to [T][Hq][128], k and v to the per-head KV buffers.
-struct EpiQkv {
+template <int EG_>
+struct EpiQkvT {
   EpiQkvArgs a;
-  static constexpr int EG = 2;  // one head of the 256-column tile per group
+  static constexpr int EG = EG_;  // one head of the tile (256 or 128 columns) per group
   // rows leave through two per-warp scratches (the head's two 64-column
   // halves), four full lines per warp store; a 4-stage ring keeps the CTA
   // near 200 KB
@@ -269,6 +275,7 @@ struct EpiQkv {
   template <int BN>
   __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, int g, bool row_ok, const PlanHdr* plan,
                                       DevStatus* st, uint8_t* scratch, int M, const Pre&) const {
+    static_assert(BN == 128 * EG, "one 128-column head per epilogue group");
     const int gc = n0 + 128 * g;
     const uint32_t base = taddr + 128 * g;
     const int lane = threadIdx.x & 31;
@@ -385,6 +392,11 @@ struct EpiQkv {
   }
 };
 
+using EpiResid = EpiResidT<2>;
+using EpiResidNarrow = EpiResidT<1>;  // 64-column tiles
+using EpiQkv = EpiQkvT<2>;
+using EpiQkvNarrow = EpiQkvT<1>;      // 128-column tiles
+
 // ---------------------------------------------------------------------------
 // the kernel, per CTA of a pair: warp 0 TMA producer, warp 1 TMEM allocation
 // and (leader only) the MMA issuer, warps 2 .. 2 + 4*EG - 1 epilogue (group
@@ -418,6 +430,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 128 * Epi::EG, 
   const int kblocks = Kdim / kBK;
   const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
 
+  pdl_launch_dependents();
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
@@ -431,9 +444,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 128 * Epi::EG, 
     }
     mbar_init(drain, 1);
     fence_barrier_init();
-    // a bounded wait already gave up in an earlier launch: the pair skips its
-    // work, on the leader's reading of the flag so both CTAs agree
-    if (leader) *skip_flag = (*reinterpret_cast<volatile const uint32_t*>(&st->flags) & ERR_WAIT_TIMEOUT) ? 1u : 0u;
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(tmem_holder), C::TMEM_COLS);
@@ -443,6 +453,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 128 * Epi::EG, 
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // everything below reads what the previous kernels wrote
+  pdl_wait();
+  // a bounded wait already gave up in an earlier launch: the pair skips its
+  // work, on the leader's reading of the flag so both CTAs agree
+  if (threadIdx.x == 0 && leader)
+    *skip_flag = (*reinterpret_cast<volatile const uint32_t*>(&st->flags) & ERR_WAIT_TIMEOUT) ? 1u : 0u;
+  cluster_sync();
   const bool skip = ld_shared_cluster_u32(map_to_rank(smem_u32(skip_flag), 0)) != 0;
 
   if (!skip) {
@@ -603,32 +620,41 @@ bool make_tmap_f16_3d(CUtensorMap* map, const void* base, const uint64_t dims[3]
   return true;
 }
 
+template <int BN, class Epi>
+static cudaError_t set_smem() {
+  return cudaFuncSetAttribute(gemm_tc_kernel<BN, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              TcCfg<BN, Epi>::SMEM);
+}
+
+template <int BN, class Epi>
+static cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
+                          const Epi& e, DevStatus* st, int grid, cudaStream_t s, bool pdl) {
+  return launch_ex(gemm_tc_kernel<BN, Epi>, dim3(grid), dim3(64 + 128 * Epi::EG), TcCfg<BN, Epi>::SMEM, s, pdl, a, b,
+                   K, N, plan, e, st);
+}
+
 cudaError_t gemm_tc_setup() {
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(gemm_tc_kernel<256, EpiResid>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                TcCfg<256, EpiResid>::SMEM)) != cudaSuccess)
+  if ((e = set_smem<256, EpiResid>()) != cudaSuccess || (e = set_smem<kNarrowResid, EpiResidNarrow>()) != cudaSuccess ||
+      (e = set_smem<256, EpiSwiglu>()) != cudaSuccess || (e = set_smem<256, EpiQkv>()) != cudaSuccess ||
+      (e = set_smem<kNarrowQkv, EpiQkvNarrow>()) != cudaSuccess)
     return e;
-  if ((e = cudaFuncSetAttribute(gemm_tc_kernel<256, EpiSwiglu>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                TcCfg<256, EpiSwiglu>::SMEM)) != cudaSuccess)
-    return e;
-  return cudaFuncSetAttribute(gemm_tc_kernel<256, EpiQkv>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              TcCfg<256, EpiQkv>::SMEM);
+  return cudaSuccess;
 }
 
 cudaError_t gemm_tc_resid(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
-                          EpiResidArgs e, DevStatus* st, int grid, cudaStream_t s) {
-  gemm_tc_kernel<256, EpiResid><<<grid, 64 + 128 * EpiResid::EG, TcCfg<256, EpiResid>::SMEM, s>>>(a, b, K, N, plan, EpiResid{e}, st);
-  return cudaGetLastError();
+                          EpiResidArgs e, DevStatus* st, int grid, cudaStream_t s, bool narrow, bool pdl) {
+  return narrow ? launch<kNarrowResid>(a, b, K, N, plan, EpiResidNarrow{e}, st, grid, s, pdl)
+                : launch<256>(a, b, K, N, plan, EpiResid{e}, st, grid, s, pdl);
 }
 cudaError_t gemm_tc_swiglu(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
-                           EpiSwigluArgs e, DevStatus* st, int grid, cudaStream_t s) {
-  gemm_tc_kernel<256, EpiSwiglu><<<grid, 64 + 128 * EpiSwiglu::EG, TcCfg<256, EpiSwiglu>::SMEM, s>>>(a, b, K, N, plan, EpiSwiglu{e}, st);
-  return cudaGetLastError();
+                           EpiSwigluArgs e, DevStatus* st, int grid, cudaStream_t s, bool pdl) {
+  return launch<256>(a, b, K, N, plan, EpiSwiglu{e}, st, grid, s, pdl);
 }
 cudaError_t gemm_tc_qkv(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
-                        EpiQkvArgs e, DevStatus* st, int grid, cudaStream_t s) {
-  gemm_tc_kernel<256, EpiQkv><<<grid, 64 + 128 * EpiQkv::EG, TcCfg<256, EpiQkv>::SMEM, s>>>(a, b, K, N, plan, EpiQkv{e}, st);
-  return cudaGetLastError();
+                        EpiQkvArgs e, DevStatus* st, int grid, cudaStream_t s, bool narrow, bool pdl) {
+  return narrow ? launch<kNarrowQkv>(a, b, K, N, plan, EpiQkvNarrow{e}, st, grid, s, pdl)
+                : launch<256>(a, b, K, N, plan, EpiQkv{e}, st, grid, s, pdl);
 }
 
 }  // namespace duolm

@@ -52,12 +52,20 @@ bool make_tmap_f16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64
 bool make_tmap_f16_3d(CUtensorMap* map, const void* base, const uint64_t dims[3], const uint64_t strides_bytes[2],
                       const uint32_t box[3], char* err, size_t errlen);
 cudaError_t gemm_tc_setup();
+// Tile widths: 256 columns, or the narrow widths for small batches (the
+// weight's tensor map must have boxes of BN / 2 rows: 32 for the residual
+// projections, 64 for QKV).
+constexpr int kNarrowResid = 64;
+constexpr int kNarrowQkv = 128;
+// pdl: launched with programmatic dependent launch (the kernel waits for its
+// predecessor itself; see pdl_wait)
 cudaError_t gemm_tc_resid(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
-                          EpiResidArgs e, DevStatus* st, int grid, cudaStream_t s);
+                          EpiResidArgs e, DevStatus* st, int grid, cudaStream_t s, bool narrow = false,
+                          bool pdl = false);
 cudaError_t gemm_tc_swiglu(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
-                           EpiSwigluArgs e, DevStatus* st, int grid, cudaStream_t s);
+                           EpiSwigluArgs e, DevStatus* st, int grid, cudaStream_t s, bool pdl = false);
 cudaError_t gemm_tc_qkv(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
-                        EpiQkvArgs e, DevStatus* st, int grid, cudaStream_t s);
+                        EpiQkvArgs e, DevStatus* st, int grid, cudaStream_t s, bool narrow = false, bool pdl = false);
 
 // ---- fp32 SIMT GEMM (the fp32 path): C = A * B^T, store or residual add.
 cudaError_t gemm_simt(const float* A, const float* B, float* C, int K, int N, int ldc, bool accumulate,
@@ -71,12 +79,12 @@ cudaError_t embed_norm(const PlanHdr* plan, const void* embed, bool embed_bf16, 
 // fp16 path: gather into x, write fp16(x * gain) and the row's sum of x^2
 cudaError_t embed_gain(const PlanHdr* plan, const void* embed, const __half* table, int64_t n_table, int vocab, int d,
                        const float* gain, float* x, __half* xg, float* ssp, int n_slots, DevStatus* st, int max_rows,
-                       cudaStream_t s);
+                       cudaStream_t s, bool pdl = false);
 template <typename OutT>
 cudaError_t rmsnorm_rows(const PlanHdr* plan, const float* x, int d, const float* gain, float eps, OutT* xn,
                          DevStatus* st, int max_rows, cudaStream_t s);
 cudaError_t score_head(const PlanHdr* plan, const float* x, int d, const float* gain, const float* w, float eps,
-                       float* scores, int max_cand, cudaStream_t s);
+                       float* scores, int max_cand, cudaStream_t s, bool pdl = false);
 cudaError_t qkv_post_f32(const PlanHdr* plan, const float* qkv, int n_q_heads, int n_kv_heads, int hd,
                          const float* gq, const float* gk, float eps, const float2* rope, int max_pos, float* q,
                          float* kc, float* vc, int64_t kv_rows, DevStatus* st, int max_rows, cudaStream_t s);
@@ -99,13 +107,13 @@ cudaError_t attention_f32(const PlanHdr* plan, const int2* reqx, const float* q,
 cudaError_t attention_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tks,
                          const CUtensorMap& tvs, const PlanHdr* plan, const int2* reqx, int64_t kv_rows,
                          int64_t store_rows, int n_q_heads, int n_kv_heads, float scale, __half* o, DevStatus* st,
-                         int grid, cudaStream_t s);
+                         int grid, cudaStream_t s, bool pdl = false);
 // KV store append: for every request r with append[r] = {n, dst} (n > 0),
 // rows [tok0_r, tok0_r + n) of this batch's K/V (every KV head) are copied
 // to store rows [dst, dst + n); row_bytes a multiple of 16
 cudaError_t kv_append(const PlanHdr* plan, const int2* append, const void* kc, const void* vc, int64_t kv_rows,
                       void* ks, void* vs, int64_t store_rows, int n_kv_heads, int row_bytes, int max_req,
-                      int grid, cudaStream_t s);
+                      int grid, cudaStream_t s, bool pdl = false);
 cudaError_t attention_tc_setup();
 // Host: the batch's attention work list {request, KV head, kind (1 branch,
 // 0 prefix), first query row} (req: {tok0, whole prefix L, K, -}; reqx: as

@@ -20,6 +20,8 @@ __global__ void kv_append_kernel(const PlanHdr* __restrict__ plan, const int2* _
                                  const uint4* __restrict__ kc, const uint4* __restrict__ vc, int64_t kv_rows,
                                  uint4* __restrict__ ks, uint4* __restrict__ vs, int64_t store_rows, int n_kv_heads,
                                  int row_words) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int n_req = plan->n_req;
   const int4* reqs = plan_array<int4>(plan, plan->off_req);
   const int64_t units = (int64_t)n_req * n_kv_heads * 2;
@@ -40,14 +42,13 @@ __global__ void kv_append_kernel(const PlanHdr* __restrict__ plan, const int2* _
 
 cudaError_t kv_append(const PlanHdr* plan, const int2* append, const void* kc, const void* vc, int64_t kv_rows,
                       void* ks, void* vs, int64_t store_rows, int n_kv_heads, int row_bytes, int max_req, int grid,
-                      cudaStream_t s) {
+                      cudaStream_t s, bool pdl) {
   if (row_bytes % 16) return cudaErrorInvalidValue;
   const int64_t units = (int64_t)max_req * n_kv_heads * 2;
   const int g = (int)std::max<int64_t>(1, std::min<int64_t>(units, grid));
-  kv_append_kernel<<<g, 256, 0, s>>>(plan, append, static_cast<const uint4*>(kc), static_cast<const uint4*>(vc),
-                                     kv_rows, static_cast<uint4*>(ks), static_cast<uint4*>(vs), store_rows,
-                                     n_kv_heads, row_bytes / 16);
-  return cudaGetLastError();
+  return launch_ex(kv_append_kernel, dim3(g), dim3(256), 0, s, pdl, plan, append, static_cast<const uint4*>(kc),
+                   static_cast<const uint4*>(vc), kv_rows, static_cast<uint4*>(ks), static_cast<uint4*>(vs),
+                   store_rows, n_kv_heads, row_bytes / 16);
 }
 
 }  // namespace duolm

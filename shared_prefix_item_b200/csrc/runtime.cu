@@ -38,6 +38,9 @@ struct LayerW {
   void* wd = nullptr;    // [d][F]
   float s_qkv = 1.f, s_o = 1.f, s_gu = 1.f, s_d = 1.f;  // 2^-shift of the fp16 copies
   CUtensorMap tm_qkv, tm_o, tm_gu, tm_d;
+  // the same weights in boxes for the narrow tiles of small batches: 32 rows
+  // (64-column tiles; qkv, o, gate/up, down) and 64 rows (QKV's 128-column tiles)
+  CUtensorMap tm_n32[4], tm_qkv_n64;
   int64_t g_attn = 0, g_q = 0, g_k = 0, g_mlp = 0;  // offsets into the gain buffer
 };
 
@@ -59,6 +62,7 @@ struct duolm_ctx {
   bool f16 = false;
   int num_sms = 148;
   int gemm_grid = 148;  // whole CTA pairs
+  bool use_pdl = true;  // programmatic dependent launch between the pass's kernels
   int qd = 0, kd = 0, group = 1, rows_per_item = 64;
 
   void* embed = nullptr;
@@ -379,6 +383,14 @@ cudaError_t launch_forward(duolm_ctx* c, int n_layers, bool with_head, int64_t* 
     __half* xg = static_cast<__half*>(c->xn);
     const int n_slots = d.d / 64;
     const float inv_d = 1.0f / (float)d.d;
+    // small batches: narrower tiles wherever 256-wide tiles would leave more
+    // than half of the CTA pairs without a tile
+    const int64_t m_tiles = (c->cap_T + 255) / 256, half_pairs = c->gemm_grid / 4;
+    const bool narrow_qkv = m_tiles * ((c->qd + 2 * c->kd) / 256) < half_pairs;
+    const bool narrow_res = m_tiles * (d.d / 256) < half_pairs;
+    // every kernel after the first may start its prologue while its
+    // predecessor finishes (it waits for the predecessor's data itself)
+    const bool pdl = c->use_pdl;
     LCK(DUOLM_PROF_EMBED, embed_gain(plan, c->embed, c->table, c->n_items, d.vocab, d.d, c->gains + c->layers[0].g_attn,
                                      c->x, xg, c->ssp, n_slots, c->status, maxT, s));
     for (int l = 0; l < n_layers; ++l) {
@@ -386,31 +398,32 @@ cudaError_t launch_forward(duolm_ctx* c, int n_layers, bool with_head, int64_t* 
       EpiQkvArgs qa{static_cast<__half*>(c->q), static_cast<__half*>(c->kc), static_cast<__half*>(c->vc), c->rope,
                     kv_rows, kMaxPos, c->gains + L.g_q, c->gains + L.g_k, L.s_qkv, d.rms_eps, c->qd, c->kd,
                     d.n_q_heads, c->ssp, n_slots, inv_d, d.rms_eps};
-      LCK(DUOLM_PROF_GEMM_QKV, gemm_tc_qkv(c->tm_xn, L.tm_qkv, d.d, c->qd + 2 * c->kd, plan, qa, c->status, c->gemm_grid, s));
+      LCK(DUOLM_PROF_GEMM_QKV, gemm_tc_qkv(c->tm_xn, narrow_qkv ? L.tm_qkv_n64 : L.tm_qkv, d.d, c->qd + 2 * c->kd,
+                                           plan, qa, c->status, c->gemm_grid, s, narrow_qkv, pdl));
       // without a store, the batch's own maps stand in for the store maps
       // (no request has cached tokens then, so no tile reads them)
       LCK(DUOLM_PROF_ATTENTION,
           attention_tc(c->tm_q3, c->tm_kc, c->tm_vc, c->ks ? c->tm_ks[l] : c->tm_kc, c->ks ? c->tm_vs[l] : c->tm_vc,
                        plan, c->reqx, kv_rows, store_rows, d.n_q_heads, d.n_kv_heads, attn_scale,
-                       static_cast<__half*>(c->o), c->status, c->num_sms, s));
+                       static_cast<__half*>(c->o), c->status, c->num_sms, s, pdl));
       if (c->ks)
         LCK(DUOLM_PROF_KV_APPEND, kv_append(plan, c->append, c->kc, c->vc, kv_rows,
                                             static_cast<__half*>(c->ks) + l * c->layer_store_elems,
                                             static_cast<__half*>(c->vs) + l * c->layer_store_elems, store_rows,
-                                            d.n_kv_heads, d.head_dim * 2, (int)c->cap_R, 2 * c->num_sms, s));
-      LCK(DUOLM_PROF_GEMM_O, gemm_tc_resid(c->tm_oact, L.tm_o, c->qd, d.d, plan,
+                                            d.n_kv_heads, d.head_dim * 2, (int)c->cap_R, 2 * c->num_sms, s, pdl));
+      LCK(DUOLM_PROF_GEMM_O, gemm_tc_resid(c->tm_oact, narrow_res ? L.tm_n32[1] : L.tm_o, c->qd, d.d, plan,
                                            EpiResidArgs{c->x, d.d, L.s_o, xg, c->gains + L.g_mlp, c->ssp, n_slots},
-                                           c->status, c->gemm_grid, s));
+                                           c->status, c->gemm_grid, s, narrow_res, pdl));
       LCK(DUOLM_PROF_GEMM_GATE_UP,
           gemm_tc_swiglu(c->tm_xn, L.tm_gu, d.d, 2 * d.ffn, plan,
                          EpiSwigluArgs{static_cast<__half*>(c->h), d.ffn, L.s_gu, c->ssp, n_slots, inv_d, d.rms_eps},
-                         c->status, c->gemm_grid, s));
+                         c->status, c->gemm_grid, s, pdl));
       const bool last = l + 1 == n_layers;
       LCK(DUOLM_PROF_GEMM_DOWN,
-          gemm_tc_resid(c->tm_h, L.tm_d, d.ffn, d.d, plan,
+          gemm_tc_resid(c->tm_h, narrow_res ? L.tm_n32[3] : L.tm_d, d.ffn, d.d, plan,
                         EpiResidArgs{c->x, d.d, L.s_d, last ? nullptr : xg,
                                      last ? nullptr : c->gains + c->layers[l + 1].g_attn, c->ssp, n_slots},
-                        c->status, c->gemm_grid, s));
+                        c->status, c->gemm_grid, s, narrow_res, pdl));
     }
   } else {
     float* xn = static_cast<float*>(c->xn);
@@ -447,7 +460,8 @@ cudaError_t launch_forward(duolm_ctx* c, int n_layers, bool with_head, int64_t* 
     }
   }
   if (with_head)
-    LCK(DUOLM_PROF_HEAD, score_head(plan, c->x, d.d, c->gains + c->g_final, c->head, d.rms_eps, c->scores, (int)c->cap_C, s));
+    LCK(DUOLM_PROF_HEAD, score_head(plan, c->x, d.d, c->gains + c->g_final, c->head, d.rms_eps, c->scores, (int)c->cap_C,
+                                    s, c->f16 && c->use_pdl));
   if (n_launch) *n_launch = launches;
   return cudaSuccess;
 }
@@ -589,7 +603,12 @@ int duolm_model_load(const duolm_model_desc* desc, const void* const* host_weigh
       if (!make_tmap_f16_2d(&L.tm_qkv, L.wqkv, D, ctx->qd + 2 * ctx->kd, 64, 128, e, sizeof e) ||
           !make_tmap_f16_2d(&L.tm_o, L.wo, ctx->qd, D, 64, 128, e, sizeof e) ||
           !make_tmap_f16_2d(&L.tm_gu, L.wgu, D, 2 * F, 64, 128, e, sizeof e) ||
-          !make_tmap_f16_2d(&L.tm_d, L.wd, F, D, 64, 128, e, sizeof e)) {
+          !make_tmap_f16_2d(&L.tm_d, L.wd, F, D, 64, 128, e, sizeof e) ||
+          !make_tmap_f16_2d(&L.tm_n32[0], L.wqkv, D, ctx->qd + 2 * ctx->kd, 64, kNarrowResid / 2, e, sizeof e) ||
+          !make_tmap_f16_2d(&L.tm_n32[1], L.wo, ctx->qd, D, 64, kNarrowResid / 2, e, sizeof e) ||
+          !make_tmap_f16_2d(&L.tm_n32[2], L.wgu, D, 2 * F, 64, kNarrowResid / 2, e, sizeof e) ||
+          !make_tmap_f16_2d(&L.tm_n32[3], L.wd, F, D, 64, kNarrowResid / 2, e, sizeof e) ||
+          !make_tmap_f16_2d(&L.tm_qkv_n64, L.wqkv, D, ctx->qd + 2 * ctx->kd, 64, kNarrowQkv / 2, e, sizeof e)) {
         fail(ctx, DUOLM_E_CUDA, "%s", e);
         return bail(DUOLM_E_CUDA);
       }
@@ -1046,6 +1065,13 @@ int duolm_score_cached(duolm_ctx* ctx, int n_requests, const int32_t* prefix_ids
   return duolm_sync(ctx);
 }
 
+int duolm_set_pdl(duolm_ctx* ctx, int enabled) {
+  if (!ctx) return DUOLM_E_ARG;
+  if (ctx->use_pdl != (enabled != 0)) invalidate_graph(ctx);
+  ctx->use_pdl = enabled != 0;
+  return 0;
+}
+
 int duolm_set_graph(duolm_ctx* ctx, int enabled) {
   if (!ctx) return DUOLM_E_ARG;
   ctx->use_graph = enabled != 0;
@@ -1132,8 +1158,10 @@ int64_t duolm_plan_bytes(const duolm_ctx* ctx) {
 }
 
 int duolm_debug_gemm(duolm_ctx* ctx, int layer, int which, const uint16_t* a, float* out) {
-  if (!ctx || !a || !out || layer < 0 || layer >= ctx->desc.n_layers || which < 0 || which > 3 || !ctx->f16)
+  if (!ctx || !a || !out || layer < 0 || layer >= ctx->desc.n_layers || which < 0 || which > 7 || !ctx->f16)
     return fail(ctx, DUOLM_E_ARG, "debug_gemm: bad arguments");
+  const bool narrow = which >= 4;  // the 64-column tiles of small batches
+  which &= 3;
   if (!ctx->prepared) return fail(ctx, DUOLM_E_STATE, "debug_gemm: nothing prepared");
   CK(cudaSetDevice(ctx->device));
   const auto& d = ctx->desc;
@@ -1142,7 +1170,8 @@ int duolm_debug_gemm(duolm_ctx* ctx, int layer, int which, const uint16_t* a, fl
   const int N = which == 0 ? ctx->qd + 2 * ctx->kd : which == 2 ? 2 * d.ffn : d.d;
   const CUtensorMap& ta = which == 1 ? ctx->tm_oact : which == 3 ? ctx->tm_h : ctx->tm_xn;
   void* abuf = which == 1 ? ctx->o : which == 3 ? ctx->h : ctx->xn;
-  const CUtensorMap& tb = which == 0 ? L.tm_qkv : which == 1 ? L.tm_o : which == 2 ? L.tm_gu : L.tm_d;
+  const CUtensorMap& tb =
+      narrow ? L.tm_n32[which] : (which == 0 ? L.tm_qkv : which == 1 ? L.tm_o : which == 2 ? L.tm_gu : L.tm_d);
   const float sc = which == 0 ? L.s_qkv : which == 1 ? L.s_o : which == 2 ? L.s_gu : L.s_d;
   const int64_t T = ctx->n_tokens;
   float* tmp = nullptr;
@@ -1152,7 +1181,7 @@ int duolm_debug_gemm(duolm_ctx* ctx, int layer, int which, const uint16_t* a, fl
   if (e == cudaSuccess)
     e = gemm_tc_resid(ta, tb, K, N, reinterpret_cast<const PlanHdr*>(ctx->plan_dev),
                       EpiResidArgs{tmp, N, sc, nullptr, nullptr, nullptr, 0},
-                      ctx->status, ctx->gemm_grid, ctx->stream);
+                      ctx->status, ctx->gemm_grid, ctx->stream, narrow);
   if (e == cudaSuccess) e = cudaMemcpyAsync(out, tmp, T * N * 4, cudaMemcpyDeviceToHost, ctx->stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(ctx->stream);
   cudaFree(tmp);

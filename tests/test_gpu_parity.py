@@ -114,10 +114,12 @@ def test_tcgen05_gemm_against_fp64(T_req):
         }
         for which, Wm in mats.items():
             A = (rng.normal(size=(T, Wm.shape[1])) * 0.5).astype(np.float16)
-            got = rk.debug_gemm(layer, which, A, Wm.shape[0])
             ref = A.astype(np.float64) @ Wm.astype(np.float64).T
-            # fp32 accumulation of K products: far inside 1e-5 of the row scale
-            assert np.abs(got - ref).max() <= 1e-5 * np.abs(ref).max(), (layer, which)
+            # 256-wide tiles (which) and the 64-wide tiles of small batches (which + 4)
+            for narrow in (0, 4):
+                got = rk.debug_gemm(layer, which + narrow, A, Wm.shape[0])
+                # fp32 accumulation of K products: far inside 1e-5 of the row scale
+                assert np.abs(got - ref).max() <= 1e-5 * np.abs(ref).max(), (layer, which, narrow)
 
 
 def test_q2_layout_mask_gather_bit_exact():
@@ -185,6 +187,25 @@ def test_graph_replay_matches_eager_and_is_deterministic():
     # gather, then per layer QKV, attention, O, gate/up, down (the norms are
     # folded into the projections), then the score head
     assert rk.launches_per_execute() == 1 + 5 * Q2.n_layers + 1
+
+
+def test_programmatic_dependent_launch_changes_no_result():
+    # each kernel after the first may start while its predecessor finishes
+    # and waits for its data itself: bit-identical scores with it on and off,
+    # graph and eager, over batches that use both tile widths
+    for seed, n_req in ((322, 3), (323, 24)):
+        wl = W.custom(Q2, Q2_ITEMS, seed, n_req, (1, 6), (3, 20), (5, 40), 1, n_instr=7)
+        rk = P.ranker(Q2, Q2_ITEMS)
+        out = []
+        for pdl in (True, False):
+            rk.set_pdl(pdl)
+            for graph in (True, False):
+                rk.set_graph(graph)
+                out.append(rk.score_workload(wl))
+        rk.set_pdl(True)
+        rk.set_graph(True)
+        for o in out[1:]:
+            assert np.array_equal(out[0], o)
 
 
 def test_host_validation_errors():
