@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--config c64|c1|stress|catalog-c64|catalog-c8|catalog-c1]
-                    [--mode mis|independent] [--reuse append|rescore] [--no-graph] [--skip-cpu]
+                    [--mode mis|independent] [--reuse append|rescore|template] [--no-graph] [--skip-cpu]
                     [--profile-steps N]
 
 One step is one pass of the whole hot path (virtual-id gather, 28 decoder
@@ -23,7 +23,9 @@ instead, one request of the same workload per step.
 request's prefix up to its last history item beforehand, and every step
 appends that item and the header (the new history arrives) before scoring;
 `rescore` stores the whole prefix and every step scores the K candidates
-only.  The scores are those of the full sequences either way.
+only; `template` stores the instruction every prompt starts with in one
+slot that all requests read.  The scores are those of the full sequences in
+every case.
 """
 from __future__ import annotations
 
@@ -139,8 +141,27 @@ class Reuse:
         elif kind == "rescore":
             self.cached = [r.L for r in wl.requests]
             keep = [0] * R
+        elif kind == "template":
+            # one slot holds the instruction every prompt starts with; every
+            # request reads it (exact cross-request reuse of a common prefix)
+            n_instr = len(wl.template.instr)
+            assert all(np.array_equal(r.prefix_ids[:n_instr], wl.template.instr) for r in wl.requests)
+            self.cached = [n_instr] * R
+            keep = [0] * R
+            r0 = wl.requests[0]
+            self.slot_tokens = n_instr
+            self.warm = (np.asarray(wl.template.instr, np.int32), np.array([0, n_instr]), r0.branch_ids.reshape(-1),
+                         np.array([0, r0.K]), wl.branch_len, np.array([0]), np.zeros(1), np.array([n_instr]))
+            new_ids = np.concatenate([r.prefix_ids[n_instr:] for r in wl.requests])
+            new_off = np.cumsum([0] + [r.L - n_instr for r in wl.requests])
+            self.step = (new_ids, new_off, b, co, wl.branch_len, np.zeros(R, np.int64), self.cached, keep)
+            self.n_slots = 1
+            self.note = (f"template: the {n_instr}-token instruction of every request read from one shared KV slot, "
+                         f"{int(new_off[-1])} new prefix tokens per step")
+            return
         else:
             raise SystemExit(f"unknown --reuse {kind}")
+        self.n_slots = R
         warm_ids = np.concatenate([r.prefix_ids[:c] for r, c in zip(wl.requests, self.cached)])
         warm_off = np.cumsum([0] + self.cached)
         new_ids = np.concatenate([r.prefix_ids[c:] for r, c in zip(wl.requests, self.cached)])
@@ -627,7 +648,7 @@ def run_ours(args, rank: int, world: int, local_rank: int, dev=None) -> None:
         if mode != S.MODE_MIS:
             raise SystemExit("--reuse needs --mode mis")
         reuse = Reuse(wl, args.reuse)
-        rk.kv_store_reserve(len(wl.requests), reuse.slot_tokens)
+        rk.kv_store_reserve(reuse.n_slots, reuse.slot_tokens)
         rk.score_cached(*reuse.warm)
 
         def prepare():
@@ -806,7 +827,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="c64")
     ap.add_argument("--mode", choices=["mis", "independent"], default="mis")
-    ap.add_argument("--reuse", choices=["append", "rescore"], default=None,
+    ap.add_argument("--reuse", choices=["append", "rescore", "template"], default=None,
                     help="score from a prefix KV store (see the module docstring)")
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")

@@ -211,3 +211,29 @@ def test_c64_history_append_matches_full_recompute():
     finally:
         rk.kv_store_reserve(0, 0)
 
+
+
+@pytest.mark.parametrize("store_ranker", [TINY, Q2], indirect=True, ids=["fp32", "bf16"])
+def test_every_request_reads_one_shared_template_slot(store_ranker):
+    # the instruction every prompt of a recipe starts with, stored once and
+    # read by all requests of a batch (the exact part of cross-request prefix
+    # sharing, Summary page 未来方向 (5)): every score equals the oracle's over
+    # the whole prefix
+    shape, rk = store_ranker
+    wl = W.custom(shape, ITEMS[shape], 341, 5, (1, 6), (3, 20), (5, 40), 1, n_instr=40, n_header=3)
+    n = 40
+    r0 = wl.requests[0]
+    for r in wl.requests:
+        assert np.array_equal(r.prefix_ids[:n], r0.prefix_ids[:n])
+    # store the instruction in slot 3 (scoring request 0's candidates once)
+    _one(rk, r0.prefix_ids[:n], r0.branch_ids, 1, 3, 0, n)
+    assert rk.kv_slot_length(3) == n
+    new = np.concatenate([r.prefix_ids[n:] for r in wl.requests])
+    off = np.cumsum([0] + [r.L - n for r in wl.requests])
+    _, _, b, co = wl.packed()
+    R_ = len(wl.requests)
+    got = P.split_scores(wl, rk.score_cached(new, off, b, co, 1, [3] * R_, [n] * R_, [0] * R_))
+    assert rk.kv_slot_length(3) == n  # read only
+    for q, r in enumerate(wl.requests):
+        ref = _oracle(shape, r.prefix_ids, r.branch_ids)
+        P.assert_scores_match(shape, got[q], ref, f"request {q}")
