@@ -315,17 +315,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const bool valid = rl < m.nrows;
       __half* dst = o + (((int64_t)m.qbase + m.q0 + rl) * n_q_heads + m.kvh * G + (r % G)) * kHD;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(tO + 32 * c, v);
+      {
+        // all 128 columns in one batch of TMEM loads (the S registers are
+        // free by now), then the row out in 32-byte stores (one full sector
+        // each)
+        uint32_t ov[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32_async(tO + 32 * c, ov[c]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) tmem_ld_fence(ov[c][j]);
         if (valid) {
-          uint32_t pw[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) pw[j] = pack_half2(v[2 * j] * inv, v[2 * j + 1] * inv);
-          uint4* p = reinterpret_cast<uint4*>(dst + 32 * c);
+          for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int q = 0; q < 4; ++q) p[q] = make_uint4(pw[4 * q], pw[4 * q + 1], pw[4 * q + 2], pw[4 * q + 3]);
+            for (int h = 0; h < 2; ++h) {
+              uint32_t w[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                w[j] = pack_half2(__uint_as_float(ov[c][16 * h + 2 * j]) * inv,
+                                  __uint_as_float(ov[c][16 * h + 2 * j + 1]) * inv);
+              st_global_v8(dst + 32 * c + 16 * h, w);
+            }
         }
       }
       tc_fence_before();
