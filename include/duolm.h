@@ -417,8 +417,9 @@ int64_t duolm_plan_bytes(const duolm_ctx *ctx);
  * One projection of layer `layer` through the tensor-core GEMM alone
  * (BF16 models only): out = a * W^T with W = wqkv (which 0, [qd+2kd][d]),
  * wo (1, [d][qd]), gate/up (2, [2*ffn][d], rows in 128-row blocks alternating
- * gate and up) or w_down (3, [d][ffn]); which + 4 runs the same product
- * with the 64-column tiles small batches use.  a: host uint16 fp16 bit patterns
+ * gate and up) or w_down (3, [d][ffn]); which + 4 computes the same product
+ * as four K-slices summed by the split-K reduction small batches use for the
+ * O and down projections.  a: host uint16 fp16 bit patterns
  * [n_tokens][K] where n_tokens is the prepared batch's token count; out: host
  * float [n_tokens][N].  Overwrites the batch's activations.  Synchronous.
  */

@@ -252,6 +252,12 @@ __device__ __forceinline__ void tma_load_3d(const CUtensorMap* map, uint32_t dst
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
+// Bring a tile of a tensor into L2 (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
+}
 // Make this thread's generic-proxy shared-memory writes visible to the async
 // proxy (TMA, tensor cores) before signalling a consumer.
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {

@@ -37,7 +37,7 @@ constexpr int kBK = 64;  // one 128-byte swizzle row of fp16
 // an A row block and it is read from DRAM once.
 // An epilogue may ask for shared-memory scratch per epilogue warp (then the
 // ring is shallower, so the CTA stays near 197 KB of shared memory).
-// Narrower tiles (BN 64 or 128, one epilogue group) serve small batches,
+// Narrower QKV tiles (BN 128, one epilogue group) serve small batches,
 // where 256-wide tiles leave most CTA pairs without work; their smaller
 // stages let the ring hold more k-blocks in the same shared memory.
 template <int BN, class Epi>
@@ -131,7 +131,7 @@ struct EpiResidT {
   }
   template <int BN>
   __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, int g, bool, const PlanHdr*, DevStatus* st,
-                                      uint8_t* scratch, int M, const Pre&) const {
+                                      uint8_t* scratch, int M, const Pre&, int) const {
     constexpr int W = BN / EG;
     static_assert(W % 64 == 0, "a group covers whole 64-column norm slots");
     const int lane = threadIdx.x & 31;
@@ -220,7 +220,7 @@ struct EpiSwiglu {
   }
   template <int BN>
   __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, int g, bool row_ok, const PlanHdr*,
-                                      DevStatus* st, uint8_t* scratch, int M, const Pre& pre) const {
+                                      DevStatus* st, uint8_t* scratch, int M, const Pre& pre, int) const {
     constexpr int H = BN / 2;   // gate columns [0, H), up columns [H, BN)
     constexpr int W = H / EG;   // outputs of this group: one 128-byte fp16 row segment
     static_assert(W == 64, "one warp store per group");
@@ -274,7 +274,7 @@ struct EpiQkvT {
   }
   template <int BN>
   __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, int g, bool row_ok, const PlanHdr* plan,
-                                      DevStatus* st, uint8_t* scratch, int M, const Pre&) const {
+                                      DevStatus* st, uint8_t* scratch, int M, const Pre&, int) const {
     static_assert(BN == 128 * EG, "one 128-column head per epilogue group");
     const int gc = n0 + 128 * g;
     const uint32_t base = taddr + 128 * g;
@@ -284,6 +284,19 @@ struct EpiQkvT {
     uint32_t* buf2 = buf1 + 32 * kScratchPad;
     // weight scale times the input row's RMSNorm factor
     const float sc = row_ok ? a.scale * row_rnorm(a.ssp, a.n_slots, row, a.inv_d, a.norm_eps) : 0.f;
+    // the store row this thread's token goes to (-1: none), shared with the
+    // warp's other lanes by shuffles when the rows are written out
+    int srow = -1;
+    if (a.ks && gc >= a.qd && row_ok) {
+      const int r = plan_array<int32_t>(plan, plan->off_treq)[row];
+      const int i = row - plan_array<int4>(plan, plan->off_req)[r].x;
+      const int2 ap = a.append[r];
+      if (i >= 0 && i < ap.x) srow = ap.y + i;
+    }
+    auto store_dst = [&](__half* base_, int head_, int r, int col) -> uint4* {
+      const int sr = __shfl_sync(0xffffffffu, srow, r);
+      return sr >= 0 ? reinterpret_cast<uint4*>(base_ + ((int64_t)head_ * a.store_rows + sr) * 128 + col) : nullptr;
+    };
     if (gc >= a.qd + a.kd) {  // value head
       const int head = (gc - a.qd - a.kd) >> 7;
 #pragma unroll 1
@@ -306,6 +319,7 @@ struct EpiQkvT {
           return rr < M ? reinterpret_cast<uint4*>(a.vc + ((int64_t)head * a.kv_rows + rr) * 128 + 64 * half)
                         : nullptr;
         });
+        if (a.ks) warp_flush_rows_128B(buf1, [&](int r) -> uint4* { return store_dst(a.vs, head, r, 64 * half); });
       }
       return;
     }
@@ -389,11 +403,49 @@ struct EpiQkvT {
       const int rr = row0 + r;
       return rr < M ? reinterpret_cast<uint4*>(dst(rr) + 64) : nullptr;
     });
+    if (a.ks && !is_q) {
+      warp_flush_rows_128B(buf1, [&](int r) -> uint4* { return store_dst(a.ks, head, r, 0); });
+      warp_flush_rows_128B(buf2, [&](int r) -> uint4* { return store_dst(a.ks, head, r, 64); });
+    }
+  }
+};
+
+// Split-K slice: the fp32 accumulator rows to the workspace, 32-byte stores.
+struct EpiPartial {
+  EpiPartialArgs a;
+  static constexpr int EG = 2;
+  static constexpr int STAGES = 6;
+  static constexpr int SCRATCH_PER_WARP = 0;
+  struct Pre {};
+  template <int BN>
+  __device__ __forceinline__ Pre prefetch(int, int, int, bool, const PlanHdr*, DevStatus*) const {
+    return Pre{};
+  }
+  template <int BN>
+  __device__ __forceinline__ void run(uint32_t taddr, int row, int n0, int g, bool row_ok, const PlanHdr*,
+                                      DevStatus*, uint8_t*, int, const Pre&, int split) const {
+    constexpr int W = BN / EG;
+    float* dst = a.ws + ((int64_t)split * a.ws_rows + row) * a.ldw + n0 + g * W;
+#pragma unroll 1
+    for (int c = 0; c < W; c += 32) {
+      uint32_t v[32];
+      tmem_ld32_async(taddr + g * W + c, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) tmem_ld_fence(v[j]);
+      if (row_ok) {
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const uint32_t w[8] = {v[8 * h], v[8 * h + 1], v[8 * h + 2], v[8 * h + 3],
+                                 v[8 * h + 4], v[8 * h + 5], v[8 * h + 6], v[8 * h + 7]};
+          st_global_v8(dst + c + 8 * h, w);
+        }
+      }
+    }
   }
 };
 
 using EpiResid = EpiResidT<2>;
-using EpiResidNarrow = EpiResidT<1>;  // 64-column tiles
 using EpiQkv = EpiQkvT<2>;
 using EpiQkvNarrow = EpiQkvT<1>;      // 128-column tiles
 
@@ -406,7 +458,7 @@ using EpiQkvNarrow = EpiQkvT<1>;      // 128-column tiles
 template <int BN, class Epi>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 128 * Epi::EG, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int Kdim,
-                   int N, const PlanHdr* __restrict__ plan, const Epi epi, DevStatus* st) {
+                   int N, const PlanHdr* __restrict__ plan, const Epi epi, DevStatus* st, int splits) {
   using C = TcCfg<BN, Epi>;
   constexpr int EG = Epi::EG;
   extern __shared__ uint8_t smem_raw[];
@@ -428,6 +480,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 128 * Epi::EG, 
   const int n_tiles = N / BN;
   const int num_tiles = m_tiles * n_tiles;
   const int kblocks = Kdim / kBK;
+  // work units: (tile, k-slice) pairs; with splits > 1 each unit sums a
+  // slice of K and the epilogue stores that partial (split-K for batches too
+  // small to give every CTA pair a tile of its own)
+  const int num_units = num_tiles * splits;
   const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
 
   pdl_launch_dependents();
@@ -444,6 +500,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 128 * Epi::EG, 
     }
     mbar_init(drain, 1);
     fence_barrier_init();
+    // the weight blocks of this CTA's first stages into L2 while the previous
+    // kernel finishes (weights are never written during a pass, so this may
+    // run before the wait for the predecessor)
+    if (pair < num_units) {
+      const int split = pair % splits, n_blk = (pair / splits) % n_tiles;
+      const int kb0 = split * kblocks / splits, kb1 = min((split + 1) * kblocks / splits, kb0 + C::STAGES);
+      for (int kb = kb0; kb < kb1; ++kb) tma_prefetch_2d(&tmB, kb * kBK, n_blk * BN + (int)rank * (BN / 2));
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(tmem_holder), C::TMEM_COLS);
@@ -468,9 +532,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 128 * Epi::EG, 
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
-        for (int tile = pair; tile < num_tiles && ok; tile += n_pairs) {
+        for (int u = pair; u < num_units && ok; u += n_pairs) {
+          const int tile = u / splits, split = u % splits;
           const int m_blk = tile / n_tiles, n_blk = tile % n_tiles;
-          for (int kb = 0; kb < kblocks; ++kb) {
+          for (int kb = split * kblocks / splits; kb < (split + 1) * kblocks / splits; ++kb) {
             if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, st, 1)) {
               ok = false;
               break;
@@ -495,13 +560,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 128 * Epi::EG, 
         uint32_t phase = 0;
         int local = 0;
         bool ok = true;
-        for (int tile = pair; tile < num_tiles && ok; tile += n_pairs, ++local) {
+        for (int u = pair; u < num_units && ok; u += n_pairs, ++local) {
+          const int split = u % splits;
+          const int kb0 = split * kblocks / splits, kb1 = (split + 1) * kblocks / splits;
           const int acc = local & 1;
           const uint32_t use = (uint32_t)(local >> 1);
           if (!mbar_wait(tempty0 + 8 * acc, (use & 1u) ^ 1u, st, 2)) break;
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + acc * BN;
-          for (int kb = 0; kb < kblocks; ++kb) {
+          for (int kb = kb0; kb < kb1; ++kb) {
             if (!mbar_wait(full0 + 8 * stage, phase, st, 3)) {
               ok = false;
               break;
@@ -512,7 +579,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 128 * Epi::EG, 
 #pragma unroll
             for (int k = 0; k < kBK / 16; ++k) {
               tc_mma_f16_pair(d_tmem, smem_desc_sw128(sa + 32 * k), smem_desc_sw128(sb + 32 * k), C::IDESC,
-                              (kb | k) != 0 ? 1u : 0u);
+                              (kb != kb0 || k != 0) ? 1u : 0u);
             }
             tc_commit_pair_both(empty0 + 8 * stage);
             if (++stage == C::STAGES) {
@@ -530,7 +597,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 128 * Epi::EG, 
       const int q4 = warp & 3;            // TMEM lane quadrant this warp may access
       const int group = (warp - 2) >> 2;  // column group of the tile
       int local = 0;
-      for (int tile = pair; tile < num_tiles; tile += n_pairs, ++local) {
+      for (int u = pair; u < num_units; u += n_pairs, ++local) {
+        const int tile = u / splits, split = u % splits;
         const int acc = local & 1;
         const uint32_t use = (uint32_t)(local >> 1);
         const int m_blk = tile / n_tiles, n_blk = tile % n_tiles;
@@ -540,7 +608,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 128 * Epi::EG, 
         tc_fence_after();
         const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q4 * 32) << 16);
         epi.template run<BN>(taddr, row, n_blk * BN, group, row < M, plan, st,
-                             smem + C::EPI_OFF + (warp - 2) * Epi::SCRATCH_PER_WARP, M, pre);
+                             smem + C::EPI_OFF + (warp - 2) * Epi::SCRATCH_PER_WARP, M, pre, split);
         // the accumulator may be overwritten once every epilogue thread of
         // the pair has read it; the reads are ordered by the tcgen05 fence,
         // the global stores need no ordering with the MMA
@@ -628,25 +696,81 @@ static cudaError_t set_smem() {
 
 template <int BN, class Epi>
 static cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
-                          const Epi& e, DevStatus* st, int grid, cudaStream_t s, bool pdl) {
+                          const Epi& e, DevStatus* st, int grid, cudaStream_t s, bool pdl, int splits = 1) {
   return launch_ex(gemm_tc_kernel<BN, Epi>, dim3(grid), dim3(64 + 128 * Epi::EG), TcCfg<BN, Epi>::SMEM, s, pdl, a, b,
-                   K, N, plan, e, st);
+                   K, N, plan, e, st, splits);
 }
 
 cudaError_t gemm_tc_setup() {
   cudaError_t e;
-  if ((e = set_smem<256, EpiResid>()) != cudaSuccess || (e = set_smem<kNarrowResid, EpiResidNarrow>()) != cudaSuccess ||
+  if ((e = set_smem<256, EpiResid>()) != cudaSuccess ||
       (e = set_smem<256, EpiSwiglu>()) != cudaSuccess || (e = set_smem<256, EpiQkv>()) != cudaSuccess ||
-      (e = set_smem<kNarrowQkv, EpiQkvNarrow>()) != cudaSuccess)
+      (e = set_smem<kNarrowQkv, EpiQkvNarrow>()) != cudaSuccess || (e = set_smem<256, EpiPartial>()) != cudaSuccess)
     return e;
   return cudaSuccess;
 }
 
 cudaError_t gemm_tc_resid(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
-                          EpiResidArgs e, DevStatus* st, int grid, cudaStream_t s, bool narrow, bool pdl) {
-  return narrow ? launch<kNarrowResid>(a, b, K, N, plan, EpiResidNarrow{e}, st, grid, s, pdl)
-                : launch<256>(a, b, K, N, plan, EpiResid{e}, st, grid, s, pdl);
+                          EpiResidArgs e, DevStatus* st, int grid, cudaStream_t s, bool pdl) {
+  return launch<256>(a, b, K, N, plan, EpiResid{e}, st, grid, s, pdl);
 }
+cudaError_t gemm_tc_partial(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
+                            EpiPartialArgs e, DevStatus* st, int grid, cudaStream_t s, int splits, bool pdl) {
+  if (splits < 1 || splits > K / kBK) return cudaErrorInvalidValue;
+  return launch<256>(a, b, K, N, plan, EpiPartial{e}, st, grid, s, pdl, splits);
+}
+
+// One CTA per row: x += scale * (sum of the split slices, in slice order),
+// then fp16(x * g_next) and the per-64-column sums of x^2 (one writer per
+// slot), the same outputs as the residual epilogue.  N a multiple of 128.
+__global__ void __launch_bounds__(256) resid_reduce_kernel(const PlanHdr* __restrict__ plan,
+                                                           const float* __restrict__ ws, int64_t ws_rows, int splits,
+                                                           EpiResidArgs e, int N, DevStatus* st) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int M = plan->n_tokens;
+  for (int r = blockIdx.x; r < M; r += gridDim.x) {
+    for (int c = 4 * threadIdx.x; c < N; c += 4 * blockDim.x) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int sp = 0; sp < splits; ++sp) {
+        const float4 v = *reinterpret_cast<const float4*>(ws + ((int64_t)sp * ws_rows + r) * N + c);
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      float4* xp = reinterpret_cast<float4*>(e.x + (int64_t)r * e.ldx + c);
+      float4 t = *xp;
+      t.x += acc.x * e.scale;
+      t.y += acc.y * e.scale;
+      t.z += acc.z * e.scale;
+      t.w += acc.w * e.scale;
+      *xp = t;
+      if (e.xg) {
+        const float4 gn = *reinterpret_cast<const float4*>(e.g_next + c);
+        const __half2 h0 = __halves2half2(to_half_checked(t.x * gn.x, st, 24), to_half_checked(t.y * gn.y, st, 24));
+        const __half2 h1 = __halves2half2(to_half_checked(t.z * gn.z, st, 24), to_half_checked(t.w * gn.w, st, 24));
+        *reinterpret_cast<uint2*>(e.xg + (int64_t)r * e.ldx + c) =
+            make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
+        // the 16 threads of a 64-column slot sum their squares
+        float ss = t.x * t.x + t.y * t.y + t.z * t.z + t.w * t.w;
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 8);
+        if ((threadIdx.x & 15) == 0) e.ssp[(int64_t)r * e.n_slots + c / 64] = ss;
+      }
+    }
+  }
+}
+
+cudaError_t resid_reduce(const PlanHdr* plan, const float* ws, int64_t ws_rows, int splits, EpiResidArgs e, int N,
+                         DevStatus* st, int max_rows, cudaStream_t s, bool pdl) {
+  if (N % 128) return cudaErrorInvalidValue;
+  return launch_ex(resid_reduce_kernel, dim3(std::max(1, max_rows)), dim3(256), 0, s, pdl, plan, ws, ws_rows, splits, e,
+                   N, st);
+}
+
 cudaError_t gemm_tc_swiglu(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
                            EpiSwigluArgs e, DevStatus* st, int grid, cudaStream_t s, bool pdl) {
   return launch<256>(a, b, K, N, plan, EpiSwiglu{e}, st, grid, s, pdl);

@@ -22,6 +22,11 @@ struct EpiResidArgs {   // x[row][col] += scale * acc  (fp32 residual stream)
   float* ssp;           // partial sums of x^2: slot n_blk * 4 + group of the tile's columns
   int n_slots;
 };
+struct EpiPartialArgs {  // split-K: the unit's fp32 partial to ws[split][row][col]
+  float* ws;
+  int64_t ws_rows;      // rows per split slice
+  int ldw;              // columns (N)
+};
 struct EpiSwigluArgs {  // tile columns [0, BN/2) gate, [BN/2, BN) up -> h = silu(g) * u, fp16
   __half* h;
   int ldh;
@@ -45,6 +50,13 @@ struct EpiQkvArgs {     // per 128-wide head: q/k RMSNorm + RoPE, v copy; fp16 o
   const float* ssp;     // partial sums of x^2 of the input rows
   int n_slots;
   float inv_d, norm_eps;
+  // prefix KV store of this layer (null: none): a request r with
+  // append[r] = {n, dst} keeps its first n new prefix rows, whose K and V
+  // also go to store rows [dst, dst + n) ([n_kv_heads][store_rows][128])
+  __half* ks;
+  __half* vs;
+  int64_t store_rows;
+  const int2* append;
 };
 
 bool make_tmap_f16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
@@ -52,16 +64,21 @@ bool make_tmap_f16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64
 bool make_tmap_f16_3d(CUtensorMap* map, const void* base, const uint64_t dims[3], const uint64_t strides_bytes[2],
                       const uint32_t box[3], char* err, size_t errlen);
 cudaError_t gemm_tc_setup();
-// Tile widths: 256 columns, or the narrow widths for small batches (the
-// weight's tensor map must have boxes of BN / 2 rows: 32 for the residual
-// projections, 64 for QKV).
-constexpr int kNarrowResid = 64;
+// Tile widths: 256 columns, or 128 for QKV in small batches (the weight's
+// tensor map then has boxes of 64 rows).
 constexpr int kNarrowQkv = 128;
 // pdl: launched with programmatic dependent launch (the kernel waits for its
 // predecessor itself; see pdl_wait)
 cudaError_t gemm_tc_resid(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
-                          EpiResidArgs e, DevStatus* st, int grid, cudaStream_t s, bool narrow = false,
-                          bool pdl = false);
+                          EpiResidArgs e, DevStatus* st, int grid, cudaStream_t s, bool pdl = false);
+// Split-K projection for small batches: each of `splits` K-slices of every
+// 256 x 256 tile stores its fp32 partial (EpiPartialArgs); resid_reduce then
+// sums the slices in slice order (deterministic) and applies the residual
+// epilogue (x += scale * sum, fp16(x * g_next), x^2 slot sums).
+cudaError_t gemm_tc_partial(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
+                            EpiPartialArgs e, DevStatus* st, int grid, cudaStream_t s, int splits, bool pdl = false);
+cudaError_t resid_reduce(const PlanHdr* plan, const float* ws, int64_t ws_rows, int splits, EpiResidArgs e, int N,
+                         DevStatus* st, int max_rows, cudaStream_t s, bool pdl = false);
 cudaError_t gemm_tc_swiglu(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,
                            EpiSwigluArgs e, DevStatus* st, int grid, cudaStream_t s, bool pdl = false);
 cudaError_t gemm_tc_qkv(const CUtensorMap& a, const CUtensorMap& b, int K, int N, const PlanHdr* plan,

@@ -30,6 +30,19 @@ namespace {
 constexpr int kMaxPos = 32768;   // position ids must stay below this
 constexpr int kKvPad = 256;      // spare KV rows so the branch key tiles of an item never leave the buffer
 constexpr int kPerLayer = 11;
+constexpr int kMaxSplits = 8;    // K-slices of a split-K projection
+
+// Split-K plan of the O and down projections for a token capacity: 1 when
+// 256 x 256 tiles already give at least half of the CTA pairs a tile, else
+// as many K-slices (at most kMaxSplits, at least 4 k-blocks each) as keep
+// the work units within the pairs.
+int splitk_factor(int64_t cap_T, int d, int K, int gemm_grid) {
+  const int64_t tiles = ((cap_T + 255) / 256) * (d / 256);
+  const int pairs = gemm_grid / 2;
+  if (tiles >= pairs / 2) return 1;
+  const int64_t by_pairs = pairs / std::max<int64_t>(tiles, 1);
+  return (int)std::max<int64_t>(1, std::min<int64_t>({(int64_t)kMaxSplits, by_pairs, (int64_t)(K / 64 / 4)}));
+}
 
 struct LayerW {
   void* wqkv = nullptr;  // [qd + 2 kd][d]
@@ -38,9 +51,8 @@ struct LayerW {
   void* wd = nullptr;    // [d][F]
   float s_qkv = 1.f, s_o = 1.f, s_gu = 1.f, s_d = 1.f;  // 2^-shift of the fp16 copies
   CUtensorMap tm_qkv, tm_o, tm_gu, tm_d;
-  // the same weights in boxes for the narrow tiles of small batches: 32 rows
-  // (64-column tiles; qkv, o, gate/up, down) and 64 rows (QKV's 128-column tiles)
-  CUtensorMap tm_n32[4], tm_qkv_n64;
+  // the QKV weights in boxes of 64 rows for the 128-column tiles of small batches
+  CUtensorMap tm_qkv_n64;
   int64_t g_attn = 0, g_q = 0, g_k = 0, g_mlp = 0;  // offsets into the gain buffer
 };
 
@@ -88,6 +100,7 @@ struct duolm_ctx {
   float* qkv32 = nullptr;
   float* gu32 = nullptr;
   float* ssp = nullptr;  // fp16 path: per-row partial sums of x^2 [T][d / 64]
+  float* splitk_ws = nullptr;  // split-K slices of the O / down projections [kMaxSplits][T][d] (small batches)
   float* scores = nullptr;
   char* plan_dev = nullptr;
   char* plan_host = nullptr;
@@ -248,6 +261,7 @@ void free_workspace(duolm_ctx* c) {
   dfree(c->qkv32);
   dfree(c->gu32);
   dfree(c->ssp);
+  dfree(c->splitk_ws);
   dfree(c->scores);
   dfree(c->plan_dev);
   dfree(c->reqx);
@@ -303,6 +317,8 @@ int reserve_impl(duolm_ctx* ctx, int64_t T, int64_t R, int64_t C) {
   if ((rc = dalloc(ctx, &ctx->h, T * d.ffn * es))) return rc;
   if (ctx->f16) {
     if ((rc = dalloc(ctx, &ctx->ssp, T * (d.d / 64) * 4))) return rc;
+    if (splitk_factor(T, d.d, std::max(ctx->qd, d.ffn), ctx->gemm_grid) > 1)
+      if ((rc = dalloc(ctx, &ctx->splitk_ws, kMaxSplits * T * d.d * 4))) return rc;
   } else {
     if ((rc = dalloc(ctx, &ctx->qkv32, T * (ctx->qd + 2 * ctx->kd) * 4))) return rc;
     if ((rc = dalloc(ctx, &ctx->gu32, T * 2 * d.ffn * 4))) return rc;
@@ -387,7 +403,10 @@ cudaError_t launch_forward(duolm_ctx* c, int n_layers, bool with_head, int64_t* 
     // than half of the CTA pairs without a tile
     const int64_t m_tiles = (c->cap_T + 255) / 256, half_pairs = c->gemm_grid / 4;
     const bool narrow_qkv = m_tiles * ((c->qd + 2 * c->kd) / 256) < half_pairs;
-    const bool narrow_res = m_tiles * (d.d / 256) < half_pairs;
+    // the O and down projections of small batches: split-K (narrow tiles
+    // would re-stream the whole activation block per 64 output columns)
+    const int split_o = c->splitk_ws ? splitk_factor(c->cap_T, d.d, c->qd, c->gemm_grid) : 1;
+    const int split_d = c->splitk_ws ? splitk_factor(c->cap_T, d.d, d.ffn, c->gemm_grid) : 1;
     // every kernel after the first may start its prologue while its
     // predecessor finishes (it waits for the predecessor's data itself)
     const bool pdl = c->use_pdl;
@@ -395,9 +414,13 @@ cudaError_t launch_forward(duolm_ctx* c, int n_layers, bool with_head, int64_t* 
                                      c->x, xg, c->ssp, n_slots, c->status, maxT, s));
     for (int l = 0; l < n_layers; ++l) {
       const LayerW& L = c->layers[l];
+      // with a prefix KV store, the kept new prefix rows' K and V also go
+      // straight to their store slot from the QKV epilogue
       EpiQkvArgs qa{static_cast<__half*>(c->q), static_cast<__half*>(c->kc), static_cast<__half*>(c->vc), c->rope,
                     kv_rows, kMaxPos, c->gains + L.g_q, c->gains + L.g_k, L.s_qkv, d.rms_eps, c->qd, c->kd,
-                    d.n_q_heads, c->ssp, n_slots, inv_d, d.rms_eps};
+                    d.n_q_heads, c->ssp, n_slots, inv_d, d.rms_eps,
+                    c->ks ? static_cast<__half*>(c->ks) + l * c->layer_store_elems : nullptr,
+                    c->ks ? static_cast<__half*>(c->vs) + l * c->layer_store_elems : nullptr, store_rows, c->append};
       LCK(DUOLM_PROF_GEMM_QKV, gemm_tc_qkv(c->tm_xn, narrow_qkv ? L.tm_qkv_n64 : L.tm_qkv, d.d, c->qd + 2 * c->kd,
                                            plan, qa, c->status, c->gemm_grid, s, narrow_qkv, pdl));
       // without a store, the batch's own maps stand in for the store maps
@@ -406,24 +429,34 @@ cudaError_t launch_forward(duolm_ctx* c, int n_layers, bool with_head, int64_t* 
           attention_tc(c->tm_q3, c->tm_kc, c->tm_vc, c->ks ? c->tm_ks[l] : c->tm_kc, c->ks ? c->tm_vs[l] : c->tm_vc,
                        plan, c->reqx, kv_rows, store_rows, d.n_q_heads, d.n_kv_heads, attn_scale,
                        static_cast<__half*>(c->o), c->status, c->num_sms, s, pdl));
-      if (c->ks)
-        LCK(DUOLM_PROF_KV_APPEND, kv_append(plan, c->append, c->kc, c->vc, kv_rows,
-                                            static_cast<__half*>(c->ks) + l * c->layer_store_elems,
-                                            static_cast<__half*>(c->vs) + l * c->layer_store_elems, store_rows,
-                                            d.n_kv_heads, d.head_dim * 2, (int)c->cap_R, 2 * c->num_sms, s, pdl));
-      LCK(DUOLM_PROF_GEMM_O, gemm_tc_resid(c->tm_oact, narrow_res ? L.tm_n32[1] : L.tm_o, c->qd, d.d, plan,
-                                           EpiResidArgs{c->x, d.d, L.s_o, xg, c->gains + L.g_mlp, c->ssp, n_slots},
-                                           c->status, c->gemm_grid, s, narrow_res, pdl));
+      const EpiResidArgs o_args{c->x, d.d, L.s_o, xg, c->gains + L.g_mlp, c->ssp, n_slots};
+      if (split_o > 1) {
+        LCK(DUOLM_PROF_GEMM_O, gemm_tc_partial(c->tm_oact, L.tm_o, c->qd, d.d, plan,
+                                               EpiPartialArgs{c->splitk_ws, c->cap_T, d.d}, c->status, c->gemm_grid,
+                                               s, split_o, pdl));
+        LCK(DUOLM_PROF_GEMM_O, resid_reduce(plan, c->splitk_ws, c->cap_T, split_o, o_args, d.d, c->status, maxT, s,
+                                            pdl));
+      } else {
+        LCK(DUOLM_PROF_GEMM_O, gemm_tc_resid(c->tm_oact, L.tm_o, c->qd, d.d, plan, o_args, c->status, c->gemm_grid, s,
+                                             pdl));
+      }
       LCK(DUOLM_PROF_GEMM_GATE_UP,
           gemm_tc_swiglu(c->tm_xn, L.tm_gu, d.d, 2 * d.ffn, plan,
                          EpiSwigluArgs{static_cast<__half*>(c->h), d.ffn, L.s_gu, c->ssp, n_slots, inv_d, d.rms_eps},
                          c->status, c->gemm_grid, s, pdl));
       const bool last = l + 1 == n_layers;
-      LCK(DUOLM_PROF_GEMM_DOWN,
-          gemm_tc_resid(c->tm_h, narrow_res ? L.tm_n32[3] : L.tm_d, d.ffn, d.d, plan,
-                        EpiResidArgs{c->x, d.d, L.s_d, last ? nullptr : xg,
-                                     last ? nullptr : c->gains + c->layers[l + 1].g_attn, c->ssp, n_slots},
-                        c->status, c->gemm_grid, s, narrow_res, pdl));
+      const EpiResidArgs d_args{c->x, d.d, L.s_d, last ? nullptr : xg,
+                                last ? nullptr : c->gains + c->layers[l + 1].g_attn, c->ssp, n_slots};
+      if (split_d > 1) {
+        LCK(DUOLM_PROF_GEMM_DOWN, gemm_tc_partial(c->tm_h, L.tm_d, d.ffn, d.d, plan,
+                                                  EpiPartialArgs{c->splitk_ws, c->cap_T, d.d}, c->status,
+                                                  c->gemm_grid, s, split_d, pdl));
+        LCK(DUOLM_PROF_GEMM_DOWN, resid_reduce(plan, c->splitk_ws, c->cap_T, split_d, d_args, d.d, c->status, maxT, s,
+                                               pdl));
+      } else {
+        LCK(DUOLM_PROF_GEMM_DOWN, gemm_tc_resid(c->tm_h, L.tm_d, d.ffn, d.d, plan, d_args, c->status, c->gemm_grid, s,
+                                                pdl));
+      }
     }
   } else {
     float* xn = static_cast<float*>(c->xn);
@@ -604,10 +637,6 @@ int duolm_model_load(const duolm_model_desc* desc, const void* const* host_weigh
           !make_tmap_f16_2d(&L.tm_o, L.wo, ctx->qd, D, 64, 128, e, sizeof e) ||
           !make_tmap_f16_2d(&L.tm_gu, L.wgu, D, 2 * F, 64, 128, e, sizeof e) ||
           !make_tmap_f16_2d(&L.tm_d, L.wd, F, D, 64, 128, e, sizeof e) ||
-          !make_tmap_f16_2d(&L.tm_n32[0], L.wqkv, D, ctx->qd + 2 * ctx->kd, 64, kNarrowResid / 2, e, sizeof e) ||
-          !make_tmap_f16_2d(&L.tm_n32[1], L.wo, ctx->qd, D, 64, kNarrowResid / 2, e, sizeof e) ||
-          !make_tmap_f16_2d(&L.tm_n32[2], L.wgu, D, 2 * F, 64, kNarrowResid / 2, e, sizeof e) ||
-          !make_tmap_f16_2d(&L.tm_n32[3], L.wd, F, D, 64, kNarrowResid / 2, e, sizeof e) ||
           !make_tmap_f16_2d(&L.tm_qkv_n64, L.wqkv, D, ctx->qd + 2 * ctx->kd, 64, kNarrowQkv / 2, e, sizeof e)) {
         fail(ctx, DUOLM_E_CUDA, "%s", e);
         return bail(DUOLM_E_CUDA);
@@ -1160,7 +1189,7 @@ int64_t duolm_plan_bytes(const duolm_ctx* ctx) {
 int duolm_debug_gemm(duolm_ctx* ctx, int layer, int which, const uint16_t* a, float* out) {
   if (!ctx || !a || !out || layer < 0 || layer >= ctx->desc.n_layers || which < 0 || which > 7 || !ctx->f16)
     return fail(ctx, DUOLM_E_ARG, "debug_gemm: bad arguments");
-  const bool narrow = which >= 4;  // the 64-column tiles of small batches
+  const bool split = which >= 4;  // split-K: four K-slices summed by the reduction kernel
   which &= 3;
   if (!ctx->prepared) return fail(ctx, DUOLM_E_STATE, "debug_gemm: nothing prepared");
   CK(cudaSetDevice(ctx->device));
@@ -1170,21 +1199,33 @@ int duolm_debug_gemm(duolm_ctx* ctx, int layer, int which, const uint16_t* a, fl
   const int N = which == 0 ? ctx->qd + 2 * ctx->kd : which == 2 ? 2 * d.ffn : d.d;
   const CUtensorMap& ta = which == 1 ? ctx->tm_oact : which == 3 ? ctx->tm_h : ctx->tm_xn;
   void* abuf = which == 1 ? ctx->o : which == 3 ? ctx->h : ctx->xn;
-  const CUtensorMap& tb =
-      narrow ? L.tm_n32[which] : (which == 0 ? L.tm_qkv : which == 1 ? L.tm_o : which == 2 ? L.tm_gu : L.tm_d);
+  const CUtensorMap& tb = which == 0 ? L.tm_qkv : which == 1 ? L.tm_o : which == 2 ? L.tm_gu : L.tm_d;
   const float sc = which == 0 ? L.s_qkv : which == 1 ? L.s_o : which == 2 ? L.s_gu : L.s_d;
   const int64_t T = ctx->n_tokens;
+  constexpr int kSlices = 4;
   float* tmp = nullptr;
+  float* ws = nullptr;
   if (int rc = dalloc(ctx, &tmp, T * N * 4)) return rc;
+  if (split)
+    if (int rc = dalloc(ctx, &ws, kSlices * T * N * 4)) {
+      cudaFree(tmp);
+      return rc;
+    }
+  const PlanHdr* plan = reinterpret_cast<const PlanHdr*>(ctx->plan_dev);
+  const EpiResidArgs args{tmp, N, sc, nullptr, nullptr, nullptr, 0};
   cudaError_t e = cudaMemsetAsync(tmp, 0, T * N * 4, ctx->stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(abuf, a, T * K * 2, cudaMemcpyHostToDevice, ctx->stream);
-  if (e == cudaSuccess)
-    e = gemm_tc_resid(ta, tb, K, N, reinterpret_cast<const PlanHdr*>(ctx->plan_dev),
-                      EpiResidArgs{tmp, N, sc, nullptr, nullptr, nullptr, 0},
-                      ctx->status, ctx->gemm_grid, ctx->stream, narrow);
+  if (e == cudaSuccess && split) {
+    e = gemm_tc_partial(ta, tb, K, N, plan, EpiPartialArgs{ws, T, N}, ctx->status, ctx->gemm_grid, ctx->stream,
+                        kSlices);
+    if (e == cudaSuccess) e = resid_reduce(plan, ws, T, kSlices, args, N, ctx->status, (int)T, ctx->stream);
+  } else if (e == cudaSuccess) {
+    e = gemm_tc_resid(ta, tb, K, N, plan, args, ctx->status, ctx->gemm_grid, ctx->stream);
+  }
   if (e == cudaSuccess) e = cudaMemcpyAsync(out, tmp, T * N * 4, cudaMemcpyDeviceToHost, ctx->stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(ctx->stream);
   cudaFree(tmp);
+  if (ws) cudaFree(ws);
   if (e != cudaSuccess) return fail(ctx, DUOLM_E_CUDA, "debug_gemm: %s", cudaGetErrorString(e));
   return check_status(ctx);
 }

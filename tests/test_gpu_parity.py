@@ -115,11 +115,12 @@ def test_tcgen05_gemm_against_fp64(T_req):
         for which, Wm in mats.items():
             A = (rng.normal(size=(T, Wm.shape[1])) * 0.5).astype(np.float16)
             ref = A.astype(np.float64) @ Wm.astype(np.float64).T
-            # 256-wide tiles (which) and the 64-wide tiles of small batches (which + 4)
-            for narrow in (0, 4):
-                got = rk.debug_gemm(layer, which + narrow, A, Wm.shape[0])
+            # whole-K tiles (which) and the split-K form small batches use for
+            # the O and down projections (which + 4: four K-slices summed in order)
+            for split in (0, 4):
+                got = rk.debug_gemm(layer, which + split, A, Wm.shape[0])
                 # fp32 accumulation of K products: far inside 1e-5 of the row scale
-                assert np.abs(got - ref).max() <= 1e-5 * np.abs(ref).max(), (layer, which, narrow)
+                assert np.abs(got - ref).max() <= 1e-5 * np.abs(ref).max(), (layer, which, split)
 
 
 def test_q2_layout_mask_gather_bit_exact():
@@ -185,8 +186,9 @@ def test_graph_replay_matches_eager_and_is_deterministic():
     rk.set_graph(True)
     assert np.array_equal(a, b) and np.array_equal(a, c)
     # gather, then per layer QKV, attention, O, gate/up, down (the norms are
-    # folded into the projections), then the score head
-    assert rk.launches_per_execute() == 1 + 5 * Q2.n_layers + 1
+    # folded into the projections), then the score head; with the split-K O
+    # and down projections of small capacities, each adds its reduction
+    assert rk.launches_per_execute() in (1 + 5 * Q2.n_layers + 1, 1 + 7 * Q2.n_layers + 1)
 
 
 def test_programmatic_dependent_launch_changes_no_result():
