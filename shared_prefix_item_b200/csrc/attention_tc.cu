@@ -158,6 +158,30 @@ struct ItemStream {
   }
 };
 
+// Packed fp32 pairs (Blackwell's f32x2 forms: one instruction does the work
+// of two) and the three-input maximum, for the softmax's per-element work.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 }  // namespace
 
 template <int G>
@@ -262,7 +286,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int j = 0; j < 32; ++j) mx[j & 3] = fmaxf(mx[j & 3], __uint_as_float(sr[c][j]));
+          for (int j = 0; j < 32; j += 2)
+            mx[(j >> 1) & 3] = fmax3f(mx[(j >> 1) & 3], __uint_as_float(sr[c][j]), __uint_as_float(sr[c][j + 1]));
         const float m_new = fmaxf(m_used, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * scale_log2);
         // the O rescale uses warp-collective TMEM loads and stores: decide it
         // for the whole warp (a row that did not need it is rescaled to its
@@ -283,21 +308,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_used = m_new;
         }
         const float nmu = m_used == -INFINITY ? 0.f : -m_used;
-        // P = 2^(s scale - m) in fp16 over the first 64 columns of S
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+        // P = 2^(s scale - m) in fp16 over the first 64 columns of S (the
+        // scaling and the row sum on packed pairs)
+        const float2 sv = make_float2(scale_log2, scale_log2), nv = make_float2(nmu, nmu);
+        float2 ls2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c][j]), scale_log2, nmu));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c][j + 1]), scale_log2, nmu));
-            ls[(j >> 1) & 3] += p0 + p1;
-            pk[j / 2] = pack_half2(p0, p1);
+          for (int jj = 0; jj < 16; ++jj) {
+            const float2 x =
+                ffma2(make_float2(__uint_as_float(sr[c][2 * jj]), __uint_as_float(sr[c][2 * jj + 1])), sv, nv);
+            const float2 p = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+            ls2[jj & 1] = fadd2(ls2[jj & 1], p);
+            pk[jj] = pack_half2(p.x, p.y);
           }
           tmem_st16_async(tS + 16 * c, pk);
         }
-        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        l += (ls2[0].x + ls2[0].y) + (ls2[1].x + ls2[1].y);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(B_PFULL0 + X));
