@@ -10,7 +10,9 @@
 //   kind 0  prefix tokens [row0, row0 + 2R): causal over the prefix;
 //   kind 1  branch tokens (whole candidates): every prefix key tile, then the
 //           tiles of the item's own branch rows under the tree rule.
-// B is left out when the item's rows all fit in A.
+// B is left out when the item's rows all fit in A; a batch too small to
+// give half the CTAs an item (one or two requests) is planned with items of
+// one sub-tile (the plan's att_rows), so that twice as many CTAs take part.
 // A request may continue a cached prefix (incremental history append): its
 // first c prefix tokens were computed by an earlier call and their K/V sit
 // in a slot of the per-layer KV store; the batch holds only the tokens after
@@ -88,10 +90,10 @@ struct Item {
   }
 };
 
+// R2: tokens per item, 2R (two sub-tiles) or R (one, for small batches)
 template <int G>
-__device__ __forceinline__ Item make_item(int4 item, int4 rq, int2 rx, int b) {
+__device__ __forceinline__ Item make_item(int4 item, int4 rq, int2 rx, int b, int R2) {
   constexpr int R = kSub / G;  // tokens per sub-tile
-  constexpr int R2 = 2 * R;    // tokens per item
   Item m;
   m.c = rx.x;
   m.slot0 = rx.y;
@@ -122,12 +124,13 @@ struct ItemStream {
   const int4* reqs;
   const int2* reqx;
   int n, step, b;
+  int rows;  // tokens per item
   int it;
   int4 d1, d2, r1;  // descriptor of it + step, it + 2 step; request of it + step
   int2 x1;          // cached prefix of that request
   __device__ ItemStream(const PlanHdr* plan, const int2* reqx_, int cta, int n_ctas, int b_)
       : items(plan_array<int4>(plan, plan->off_items)), reqs(plan_array<int4>(plan, plan->off_req)), reqx(reqx_),
-        b(b_) {
+        b(b_), rows(plan->att_rows == kSub / G ? kSub / G : 2 * kSub / G) {
     if (plan->att_ctas == n_ctas) {
       const int32_t* off = plan_array<int32_t>(plan, plan->off_cta);
       it = off[cta];
@@ -147,7 +150,7 @@ struct ItemStream {
   __device__ bool valid() const { return it < n; }
   // the current item; advances the prefetch window
   __device__ Item next() {
-    const Item m = make_item<G>(d1, r1, x1, b);
+    const Item m = make_item<G>(d1, r1, x1, b, rows);
     const int4 z = make_int4(0, 0, 0, 0);
     it += step;
     d1 = d2;

@@ -46,7 +46,8 @@ struct PlanHdr {
   int32_t branch_len;   // b
   int32_t n_items;      // attention work items
   int32_t att_ctas;     // CTAs the attention work list is divided among (0: none)
-  int32_t pad1, pad2;
+  int32_t att_rows;     // query tokens per attention item (two sub-tiles, or one for small batches)
+  int32_t pad2;
   int64_t off_ids;      // int32 [T]   ranker ids
   int64_t off_pos;      // int32 [T]   position ids
   int64_t off_req;      // int4  [n_req]  {tok0, L, K, 0}

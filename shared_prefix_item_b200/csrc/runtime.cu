@@ -873,10 +873,28 @@ int prepare_impl(duolm_ctx* ctx, int n_requests, const int32_t* prefix_ids, cons
   int64_t n_items = 0;
   if (ctx->f16) {
     const int G = ctx->num_sms;
+    const int H = ctx->desc.n_kv_heads;
     std::vector<int32_t> cta_range((size_t)G + 1);
-    n_items = plan_attention(rq, rx, R, ctx->desc.n_kv_heads, ctx->rows_per_item, branch_len, G, ctx->cap_I,
+    // A batch whose items would fill at most half the CTAs (one or two
+    // requests) gets items of one query sub-tile instead of two: twice as
+    // many CTAs share the work, and each runs one softmax chain.
+    int rows = ctx->rows_per_item;
+    if (2 * branch_len <= rows) {
+      const int per = (rows / branch_len) * branch_len;
+      int64_t n_full = 0;
+      for (int64_t r = 0; r < R; ++r)
+        n_full += ((int64_t)rq[r].z * branch_len + per - 1) / per + (rq[r].y - rx[r].x + rows - 1) / rows;
+      if (2 * n_full * H <= G) rows /= 2;
+    }
+    n_items = plan_attention(rq, rx, R, H, rows, branch_len, G, ctx->cap_I,
                              reinterpret_cast<int4*>(base + hdr.off_items), cta_range.data());
+    if (n_items < 0 && rows != ctx->rows_per_item) {
+      rows = ctx->rows_per_item;
+      n_items = plan_attention(rq, rx, R, H, rows, branch_len, G, ctx->cap_I,
+                               reinterpret_cast<int4*>(base + hdr.off_items), cta_range.data());
+    }
     if (n_items < 0) return fail(ctx, DUOLM_E_CAPACITY, "prepare: work list overflow");
+    hdr.att_rows = rows;
     hdr.att_ctas = G;
     hdr.off_cta = hdr.off_items + align16(n_items * 16);
     memcpy(base + hdr.off_cta, cta_range.data(), (size_t)(G + 1) * 4);
